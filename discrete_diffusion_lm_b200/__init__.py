@@ -1,0 +1,263 @@
+"""Python binding of libdg, the B200 (sm_100a) sampler library for block-parallel
+uniform-noise discrete diffusion (DiffusionGemma Technical Report, section "Method").
+
+The binding only marshals arguments: torch tensors supply device memory and
+the current CUDA stream; every step of the computation runs in libdg's CUDA
+kernels.  There is no CPU fallback: if libdg.so is missing or the device is not
+sm_100, the calls raise.
+
+Functions carry the C ABI's names (include/dg.h):
+    dg_sampler_step, dg_selfcond, dg_forward_noise, dg_canvas_ce
+plus the workspace-size queries, dg_last_error, dg_launch_count, dg_version.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdg.so")
+
+DG_OK = 0
+DG_F32, DG_BF16 = 0, 1
+DG_SCHED = {"linear": 0, "cosine": 1}
+DG_X0 = {"sample": 0, "greedy": 1}
+DG_GUMBEL_CHUNK = 512
+DG_MAX_CANVASES = 256
+
+
+class DGError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_p, _i32, _i64, _u32, _u64, _sz, _int = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                         ctypes.c_uint64, ctypes.c_size_t, ctypes.c_int)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdg.so (built in-tree by discrete_diffusion_lm_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m discrete_diffusion_lm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.dg_last_error.restype = ctypes.c_char_p
+        L.dg_version.restype = ctypes.c_char_p
+        L.dg_launch_count.restype = _u64
+        L.dg_sampler_step_workspace_size.argtypes = [_i32, _i32]
+        L.dg_sampler_step_workspace_size.restype = _sz
+        L.dg_sampler_step.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32, _int,
+                                      _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]
+        L.dg_selfcond_workspace_size.argtypes = [_i32, _i32, _i32, _int, _int, _int]
+        L.dg_selfcond_workspace_size.restype = _sz
+        L.dg_selfcond.argtypes = [_p, _int, _i64, _i32, _i32, _i32, _p, _p, _p, _int, _i32, _p, _p, _sz, _p]
+        L.dg_forward_noise.argtypes = [_p, _i32, _i32, _i32, _i32, _i32, _int, _p, _u64, _p, _p, _p]
+        L.dg_canvas_ce_workspace_size.argtypes = [_i32, _i32, _i32]
+        L.dg_canvas_ce_workspace_size.restype = _sz
+        L.dg_canvas_ce.argtypes = [_p, _int, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _sz, _p]
+        _lib = L
+    return _lib
+
+
+def dg_last_error() -> str:
+    return lib().dg_last_error().decode()
+
+
+def dg_version() -> str:
+    return lib().dg_version().decode()
+
+
+def dg_launch_count() -> int:
+    return int(lib().dg_launch_count())
+
+
+def _check(fn: str, rc: int):
+    if rc != DG_OK:
+        raise DGError(fn, rc, dg_last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DG_BF16
+    if t.dtype == torch.float32:
+        return DG_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _row_major_2d(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit stride along the last dim")
+    return t.stride(0)
+
+
+def _host_doubles(vals: Sequence[float], n: int):
+    if len(vals) != n:
+        raise ValueError(f"expected {n} per-canvas values, got {len(vals)}")
+    return (ctypes.c_double * n)(*[float(v) for v in vals])
+
+
+def _host_floats(vals, n: int):
+    if vals is None:
+        return None
+    if len(vals) != n:
+        raise ValueError(f"expected {n} per-canvas values, got {len(vals)}")
+    return (ctypes.c_float * n)(*[float(v) for v in vals])
+
+
+def _expand(v, n):
+    if isinstance(v, (int, float)):
+        return [float(v)] * n
+    return list(v)
+
+
+# Workspaces are zero-filled once and reused: every successful call leaves their counters at
+# zero.  The layout inside a workspace depends on the call's shape, so a cached workspace is
+# zero-filled again (on the call's stream) whenever the shape it serves changes.
+_WS: dict = {}
+
+
+def workspace(kind: str, nbytes: int, device, layout=None, stream=None) -> torch.Tensor:
+    """A cached zero-filled workspace of at least nbytes for calls of shape `layout`."""
+    dev = torch.device(device)
+    key = (kind, dev.type, dev.index)
+    ws, last = _WS.get(key, (None, None))
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    elif last != layout:
+        with torch.cuda.stream(torch.cuda.current_stream(dev) if stream is None else stream):
+            ws.zero_()
+    _WS[key] = (ws, layout)
+    return ws
+
+
+def dg_sampler_step_workspace_size(rows: int, V: int) -> int:
+    return int(lib().dg_sampler_step_workspace_size(rows, V))
+
+
+def dg_selfcond_workspace_size(rows: int, V: int, d: int, logits_dtype: int, embed_dtype: int, have_lse: bool) -> int:
+    return int(lib().dg_selfcond_workspace_size(rows, V, d, logits_dtype, embed_dtype, int(bool(have_lse))))
+
+
+def dg_canvas_ce_workspace_size(n_seq: int, C: int, V: int) -> int:
+    return int(lib().dg_canvas_ce_workspace_size(n_seq, C, V))
+
+
+def dg_sampler_step(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V: Optional[int] = None,
+                    schedule: str = "cosine", inv_tau=None, seed: int = 0, step: int = 0, mode: str = "sample",
+                    out: Optional[dict] = None, ws: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """One sampler step over B = rows / C canvases.  Returns the dict of output tensors
+    (x_next, x0_hat, argmax, max_prob, lse, entropy, branch); pass `out` to reuse buffers."""
+    ld = _row_major_2d(logits, "logits")
+    R = logits.shape[0]
+    V = logits.shape[1] if V is None else V
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = logits.device
+    if out is None:
+        out = {
+            "x_next": torch.empty(R, dtype=torch.int32, device=dev),
+            "x0_hat": torch.empty(R, dtype=torch.int32, device=dev),
+            "argmax": torch.empty(R, dtype=torch.int32, device=dev),
+            "max_prob": torch.empty(R, dtype=torch.float32, device=dev),
+            "lse": torch.empty(R, dtype=torch.float32, device=dev),
+            "entropy": torch.empty(R, dtype=torch.float32, device=dev),
+            "branch": torch.empty(R, dtype=torch.uint8, device=dev),
+        }
+    nbytes = dg_sampler_step_workspace_size(R, V)
+    if ws is None:
+        ws = workspace("sampler_step", nbytes, dev, (R, V), stream)
+    rc = lib().dg_sampler_step(
+        _ptr(logits), _dtype_code(logits), ld, _ptr(x_t), B, C, V, DG_SCHED[schedule],
+        _host_doubles(_expand(t, B), B), _host_doubles(_expand(dt, B), B),
+        _host_floats(None if inv_tau is None else _expand(inv_tau, B), B),
+        ctypes.c_uint64(seed), ctypes.c_uint32(step), DG_X0[mode],
+        _ptr(out.get("x_next")), _ptr(out.get("x0_hat")), _ptr(out.get("argmax")), _ptr(out.get("max_prob")),
+        _ptr(out.get("lse")), _ptr(out.get("entropy")), _ptr(out.get("branch")),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("dg_sampler_step", rc)
+    return out
+
+
+def dg_selfcond(logits: torch.Tensor, E: torch.Tensor, C: int, *, V: Optional[int] = None, inv_tau=None,
+                lse: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """z = softmax(logits * inv_tau) @ E in bf16 (tcgen05 tensor cores)."""
+    ld = _row_major_2d(logits, "logits")
+    if E.dim() != 2 or not E.is_contiguous():
+        raise ValueError("E must be a contiguous [V, d] tensor")
+    R = logits.shape[0]
+    V = E.shape[0] if V is None else V
+    d = E.shape[1]
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = logits.device
+    if z is None:
+        z = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+    nbytes = dg_selfcond_workspace_size(R, V, d, _dtype_code(logits), _dtype_code(E), lse is not None)
+    if ws is None:
+        ws = workspace("selfcond", nbytes, dev, (R, V, d, lse is None, E.dtype), stream)
+    rc = lib().dg_selfcond(
+        _ptr(logits), _dtype_code(logits), ld, B, C, V,
+        _host_floats(None if inv_tau is None else _expand(inv_tau, B), B), _ptr(lse),
+        _ptr(E), _dtype_code(E), d, _ptr(z), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("dg_selfcond", rc)
+    return z
+
+
+def dg_forward_noise(x0: torch.Tensor, P: int, K: int, C: int, V: int, t, *, schedule: str = "cosine",
+                     seed: int = 0, x_t: Optional[torch.Tensor] = None, canvas_idx: Optional[torch.Tensor] = None,
+                     stream=None):
+    """Corrupt the K canvases of each sequence; returns (x_t, canvas_idx)."""
+    if x0.dim() != 2 or not x0.is_contiguous() or x0.dtype != torch.int32:
+        raise ValueError("x0 must be a contiguous int32 [n_seq, P + K*C] tensor")
+    n_seq = x0.shape[0]
+    if x_t is None:
+        x_t = torch.empty_like(x0)
+    if canvas_idx is None:
+        canvas_idx = torch.empty(n_seq, dtype=torch.int32, device=x0.device)
+    rc = lib().dg_forward_noise(_ptr(x0), n_seq, P, K, C, V, DG_SCHED[schedule],
+                                _host_doubles(_expand(t, n_seq), n_seq), ctypes.c_uint64(seed), _ptr(x_t),
+                                _ptr(canvas_idx), _stream(stream))
+    _check("dg_forward_noise", rc)
+    return x_t, canvas_idx
+
+
+def dg_canvas_ce(logits: torch.Tensor, x0: torch.Tensor, canvas_idx: torch.Tensor, P: int, K: int, C: int, *,
+                 V: Optional[int] = None, loss_rows=None, loss_seq=None, lse_rows=None,
+                 ws: Optional[torch.Tensor] = None, stream=None):
+    """Cross-entropy of each sequence's chosen canvas; returns (loss_rows, loss_seq, lse_rows)."""
+    ld = _row_major_2d(logits, "logits")
+    R = logits.shape[0]
+    V = logits.shape[1] if V is None else V
+    n_seq = x0.shape[0]
+    if R != n_seq * C:
+        raise ValueError("logits must have n_seq * C rows")
+    dev = logits.device
+    loss_rows = torch.empty(R, dtype=torch.float32, device=dev) if loss_rows is None else loss_rows
+    loss_seq = torch.empty(n_seq, dtype=torch.float32, device=dev) if loss_seq is None else loss_seq
+    lse_rows = torch.empty(R, dtype=torch.float32, device=dev) if lse_rows is None else lse_rows
+    nbytes = dg_canvas_ce_workspace_size(n_seq, C, V)
+    if ws is None:
+        ws = workspace("canvas_ce", nbytes, dev, (n_seq, C, V), stream)
+    rc = lib().dg_canvas_ce(_ptr(logits), _dtype_code(logits), ld, _ptr(x0), _ptr(canvas_idx), n_seq, P, K, C, V,
+                            _ptr(loss_rows), _ptr(loss_seq), _ptr(lse_rows), _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream))
+    _check("dg_canvas_ce", rc)
+    return loss_rows, loss_seq, lse_rows

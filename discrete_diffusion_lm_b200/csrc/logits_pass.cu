@@ -1,0 +1,405 @@
+// Logits pass: one streaming read of each logits row, then a per-row merge.
+//
+// DiffusionGemma Technical Report (hyper.ai summary), section "Method":
+//   p0 = Softmax(L_t / tau_t)  and  x_{t-dt} ~ Step(x_t, p0),
+// with the forward path kappa_t delta(x_t, x_0) + (1 - kappa_t)/V.  The same pass, with a different
+// epilogue, gives the log-sum-exp for the self-conditioning contraction and the canvas
+// cross-entropy L = -sum_i log p(x_0^i | ...).
+//
+// Phase 1 (all CTAs): each warp streams whole chunks of kChunk = 2048 consecutive ids of one row
+//   with 16-byte non-allocating loads (bf16: 8 loads of 16 B per lane, 512 B per warp-load),
+//   computes the chunk's raw maximum, S = sum exp(l' - m') and T = sum exp(l' - m')(l' - m') with
+//   l' = l * inv_tau and m' = max l', and writes one 16-byte record per chunk.
+// Phase 2 (the last CTA to finish a row, found by an atomic ticket -- nobody waits): merges the
+//   row's chunk records into lse, max-prob and entropy, finds the argmax, draws x0_hat by two-level
+//   Gumbel-max (level 1 over chunk records, level 2 by re-reading the winning chunk from L2), and
+//   samples the Step posterior with one Philox draw.  It leaves the ticket at zero.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dg {
+
+namespace {
+
+// bf16 -1.0e30 (0xF14A), used twice in a 32-bit word: -inf logits are clamped to it so that the
+// entropy sum never forms 0 * -inf.
+constexpr uint32_t kNegBigBf16x2 = 0xF14AF14Au;
+__device__ __forceinline__ float neg_big(bool bf16) {
+    return bf16 ? __uint_as_float(0xF14A0000u) : kNegBig;
+}
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+    __nv_bfloat162 r = __hmax2(x, y);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+struct ChunkStats {
+    float m_raw;  // max of the (clamped) raw logits in the chunk
+    float S;      // sum exp(l' - m'),            m' = m_raw * inv_tau (fp32)
+    float T;      // sum exp(l' - m') (l' - m')   (natural-log units)
+};
+
+// Reductions over the 8 lanes that share one chunk (lanes 8k .. 8k+7).
+__device__ __forceinline__ float max8(float v) {
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float sum8(float v) {
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// A chunk whose maximum is the clamp value holds only masked (-inf) logits: its mass is zero.
+// The shuffles run on every lane (the mask names the whole warp); only the result is selected.
+__device__ __forceinline__ ChunkStats finish(float m_raw, float s, float t, float nbig) {
+    ChunkStats cs;
+    cs.m_raw = m_raw;
+    const float S = sum8(s);
+    const float T = sum8(t) * kLn2;
+    const bool masked = !(m_raw > nbig);
+    cs.S = masked ? 0.f : S;
+    cs.T = masked ? 0.f : T;
+    return cs;
+}
+
+// One full group of 4 chunks (2048 ids) by one warp, bf16.  Lane l owns chunk l / 8 of the group;
+// its 8 lanes read the chunk's 1 KB as 8 loads of 16 B, each load instruction covering four
+// contiguous 128-byte segments across the warp.
+__device__ __forceinline__ ChunkStats group_full_bf16(const char* group, int lane, float inv_tau) {
+    const char* chunk = group + (lane >> 3) * (kChunk * 2) + (lane & 7) * 16;
+    uint32_t w[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 v = ld_stream_v4(chunk + i * 128);
+        w[4 * i + 0] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+    }
+    uint32_t mx = kNegBigBf16x2;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        w[i] = bmax2(w[i], kNegBigBf16x2);
+        mx = bmax2(mx, w[i]);
+    }
+    const float m_raw = max8(fmaxf(bf16_lo(mx), bf16_hi(mx)));
+    const float a = inv_tau * kLog2e;
+    const float nb = -(m_raw * inv_tau) * kLog2e;
+    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float x0 = fmaf(bf16_lo(w[i]), a, nb);
+        const float x1 = fmaf(bf16_hi(w[i]), a, nb);
+        const float e0 = ex2_approx(x0);
+        const float e1 = ex2_approx(x1);
+        s0 += e0;
+        s1 += e1;
+        t0 = fmaf(e0, x0, t0);
+        t1 = fmaf(e1, x1, t1);
+    }
+    return finish(m_raw, s0 + s1, t0 + t1, neg_big(true));
+}
+
+// Same for fp32: a chunk is 2 KB, 16 loads of 16 B per lane.
+__device__ __forceinline__ ChunkStats group_full_f32(const char* group, int lane, float inv_tau) {
+    const char* chunk = group + (lane >> 3) * (kChunk * 4) + (lane & 7) * 16;
+    float f[64];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint4 v = ld_stream_v4(chunk + i * 128);
+        f[4 * i + 0] = __uint_as_float(v.x);
+        f[4 * i + 1] = __uint_as_float(v.y);
+        f[4 * i + 2] = __uint_as_float(v.z);
+        f[4 * i + 3] = __uint_as_float(v.w);
+    }
+    float m = kNegBig;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        f[i] = fmaxf(f[i], kNegBig);
+        m = fmaxf(m, f[i]);
+    }
+    const float m_raw = max8(m);
+    const float a = inv_tau * kLog2e;
+    const float nb = -(m_raw * inv_tau) * kLog2e;
+    float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) {
+        const float x0 = fmaf(f[i], a, nb);
+        const float x1 = fmaf(f[i + 1], a, nb);
+        const float e0 = ex2_approx(x0);
+        const float e1 = ex2_approx(x1);
+        s0 += e0;
+        s1 += e1;
+        t0 = fmaf(e0, x0, t0);
+        t1 = fmaf(e1, x1, t1);
+    }
+    return finish(m_raw, s0 + s1, t0 + t1, kNegBig);
+}
+
+// A group that runs past V (the ragged tail, or V < 2048): element-wise and bounds-checked; lanes
+// whose chunk starts at or past V compute an empty chunk.
+__device__ __noinline__ ChunkStats group_ragged(const void* row, bool bf16, int32_t chunk_lo, int32_t V, int lane,
+                                               float inv_tau) {
+    const float nbig = neg_big(bf16);
+    const int32_t lo = chunk_lo + (lane >> 3) * kChunk;
+    const int32_t hi = min(lo + kChunk, V);
+    float m = nbig;
+    for (int32_t v = lo + (lane & 7); v < hi; v += 8) m = fmaxf(m, fmaxf(load_logit(row, v, bf16), nbig));
+    const float m_raw = max8(m);
+    const float a = inv_tau * kLog2e;
+    const float nb = -(m_raw * inv_tau) * kLog2e;
+    float s = 0.f, t = 0.f;
+    for (int32_t v = lo + (lane & 7); v < hi; v += 8) {
+        const float x = fmaf(fmaxf(load_logit(row, v, bf16), nbig), a, nb);
+        const float e = ex2_approx(x);
+        s += e;
+        t = fmaf(e, x, t);
+    }
+    return finish(m_raw, s, t, nbig);
+}
+
+struct MergeShared {
+    float f[kPassWarps];
+    int i[kPassWarps];
+    int flag;
+};
+
+template <bool kBf16, int kKind>
+__device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t canvas, float inv_tau,
+                                       const void* rowp, MergeShared& sh) {
+    const int tid = threadIdx.x;
+    const int32_t nch = p.n_chunks;
+    const float4* rec = p.rec + static_cast<size_t>(row) * nch;
+    const float nbig = neg_big(kBf16);
+
+    // Row statistics from the chunk records (log-sum-exp merge).
+    float mr = -INFINITY;
+    for (int32_t j = tid; j < nch; j += kPassThreads) mr = fmaxf(mr, ld_cg_f4(rec + j).x);
+    const float m_raw = block_max<kPassWarps>(mr, sh.f);
+    const float m_row = m_raw * inv_tau;
+    float s = 0.f, t = 0.f;
+    for (int32_t j = tid; j < nch; j += kPassThreads) {
+        const float4 r = ld_cg_f4(rec + j);
+        const float dm = r.x * inv_tau - m_row;
+        const float f = expf(dm);
+        s = fmaf(r.y, f, s);
+        t = fmaf(f, fmaf(r.y, dm, r.z), t);
+    }
+    const float S = block_sum<kPassWarps>(s, sh.f);
+    const float T = block_sum<kPassWarps>(t, sh.f);
+    const float ln_s = logf(S);
+    const float lse = m_row + ln_s;
+
+    if (kKind == kPassStats) {
+        if (tid == 0) {
+            p.lse[row] = lse;
+            p.row_ticket[row] = 0u;
+        }
+        return;
+    }
+
+    if (kKind == kPassCE) {
+        const int32_t b = row / p.C;
+        const int32_t i = row - b * p.C;
+        if (tid == 0) {
+            const int32_t k = p.canvas_idx[b];
+            float loss = __int_as_float(0x7fc00000);  // NaN for an out-of-range canvas or target
+            if (k >= 0 && k < p.K) {
+                const int32_t target =
+                    p.x0[static_cast<int64_t>(b) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i];
+                if (target >= 0 && target < p.V) loss = lse - load_logit(rowp, target, kBf16);
+            }
+            p.loss_rows[row] = loss;
+            if (p.lse) p.lse[row] = lse;
+            p.row_ticket[row] = 0u;
+            __threadfence();
+            const unsigned prev = atomicAdd(&p.seq_ticket[b], 1u);
+            sh.flag = prev == static_cast<unsigned>(p.C - 1);
+        }
+        __syncthreads();
+        if (!sh.flag) return;
+        __threadfence();
+        float acc = 0.f;
+        for (int32_t q = tid; q < p.C; q += kPassThreads)
+            acc += ld_cg_f(p.loss_rows + static_cast<int64_t>(b) * p.C + q);
+        const float total = block_sum<kPassWarps>(acc, sh.f);
+        if (tid == 0) {
+            if (p.loss_seq) p.loss_seq[b] = total;
+            p.seq_ticket[b] = 0u;
+        }
+        return;
+    }
+
+    // ---- sampler epilogue ----
+    // argmax: the first chunk whose raw maximum is the row maximum, then the first id in it.
+    int jm = 0x7fffffff;
+    for (int32_t j = tid; j < nch; j += kPassThreads)
+        if (ld_cg_f4(rec + j).x == m_raw) {
+            jm = j;
+            break;
+        }
+    jm = block_min_int<kPassWarps>(jm, sh.i);
+    if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
+    int am = 0x7fffffff;
+    {
+        const int32_t lo = jm * kChunk, hi = min(lo + kChunk, p.V);
+        for (int32_t v = lo + tid; v < hi; v += kPassThreads)
+            if (fmaxf(load_logit(rowp, v, kBf16), nbig) == m_raw) {
+                am = v;
+                break;
+            }
+    }
+    am = block_min_int<kPassWarps>(am, sh.i);
+    if (am >= p.V) am = jm * kChunk;
+
+    int32_t x0;
+    if (p.mode == DG_X0_GREEDY) {
+        x0 = am;
+    } else {
+        // Level 1: chunk scores lse_c + G_c; thread q scores chunks 4q .. 4q+3 from one Philox call.
+        float bs = -INFINITY;
+        int bj = 0x7fffffff;
+        for (int32_t q = tid; 4 * q < nch; q += kPassThreads) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
+                p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int32_t j = 4 * q + k;
+                if (j < nch) {
+                    const float4 r = ld_cg_f4(rec + j);
+                    const float sc = (r.x * inv_tau + logf(r.y)) + gumbel_from_word(word_of(w, k));
+                    if (sc > bs) {
+                        bs = sc;
+                        bj = j;
+                    }
+                }
+            }
+        }
+        block_argmax<kPassWarps>(bs, bj, sh.f, sh.i);
+        if (bj >= nch) bj = jm;  // NaN scores only
+        // Level 2: the ids of the winning chunk; thread q < 128 takes ids lo + 4q .. lo + 4q + 3.
+        const int32_t lo = bj * kChunk, hi = min(lo + kChunk, p.V);
+        float bs2 = -INFINITY;
+        int bv = 0x7fffffff;
+        const int32_t vg = lo + 4 * tid;
+        if (tid < kChunk / 4 && vg < hi) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(vg) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
+                p.key0, p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int32_t v = vg + k;
+                if (v < hi) {
+                    const float sc = fmaxf(load_logit(rowp, v, kBf16), nbig) * inv_tau + gumbel_from_word(word_of(w, k));
+                    if (sc > bs2) {
+                        bs2 = sc;
+                        bv = v;
+                    }
+                }
+            }
+        }
+        block_argmax<kPassWarps>(bs2, bv, sh.f, sh.i);
+        x0 = (bv >= lo && bv < hi) ? bv : am;
+    }
+
+    if (tid == 0) {
+        const int32_t xt = p.x_t[row];
+        unsigned long long t_stay, t_jump;
+        if (x0 != xt) {
+            t_stay = p.thr_stay_diff[canvas];
+            t_jump = p.thr_jump_diff[canvas];
+        } else {
+            t_stay = p.thr_stay_same[canvas];
+            t_jump = t_stay;
+        }
+        const uint4 w = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), p.step, kDomStep), p.key0, p.key1);
+        const unsigned long long u = w.x;
+        int32_t xn;
+        uint8_t br;
+        if (u < t_stay) {
+            xn = xt;
+            br = 0;
+        } else if (u < t_jump) {
+            xn = x0;
+            br = 1;
+        } else {
+            xn = word_to_index(w.y, p.V);
+            br = 2;
+        }
+        p.x_next[row] = xn;
+        if (p.x0_hat) p.x0_hat[row] = x0;
+        if (p.argmax) p.argmax[row] = am;
+        if (p.max_prob) p.max_prob[row] = 1.0f / S;
+        if (p.lse) p.lse[row] = lse;
+        if (p.entropy) p.entropy[row] = ln_s - T / S;
+        if (p.branch) p.branch[row] = br;
+        p.row_ticket[row] = 0u;
+    }
+}
+
+template <bool kBf16, int kKind>
+__global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_constant__ PassParams p) {
+    __shared__ MergeShared sh;
+    const int32_t row = blockIdx.x / p.segs;
+    const int32_t seg = blockIdx.x - row * p.segs;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t canvas = row / p.C;
+    const float inv_tau = kKind == kPassCE ? 1.0f : p.inv_tau[canvas];
+    constexpr int kElt = kBf16 ? 2 : 4;
+    const char* rowp = reinterpret_cast<const char*>(p.logits) + static_cast<size_t>(row) * p.ld * kElt;
+    float4* rec = p.rec + static_cast<size_t>(row) * p.n_chunks;
+
+    // Groups of 4 chunks (2048 ids) per warp-iteration; this CTA owns groups [g_begin, g_end).
+    const int32_t n_groups = (p.V + 4 * kChunk - 1) / (4 * kChunk);
+    const int32_t g_begin = seg * p.groups_per_cta;
+    const int32_t g_end = min(g_begin + p.groups_per_cta, n_groups);
+    for (int32_t gi = g_begin + warp; gi < g_end; gi += kPassWarps) {
+        const int32_t lo = gi * 4 * kChunk;
+        ChunkStats cs;
+        if (lo + 4 * kChunk <= p.V)
+            cs = kBf16 ? group_full_bf16(rowp + static_cast<size_t>(lo) * kElt, lane, inv_tau)
+                       : group_full_f32(rowp + static_cast<size_t>(lo) * kElt, lane, inv_tau);
+        else
+            cs = group_ragged(rowp, kBf16, lo, p.V, lane, inv_tau);
+        const int32_t c = 4 * gi + (lane >> 3);
+        if ((lane & 7) == 0 && c < p.n_chunks) rec[c] = make_float4(cs.m_raw, cs.S, cs.T, 0.f);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(&p.row_ticket[row], 1u);
+        sh.flag = prev == static_cast<unsigned>(p.segs - 1);
+    }
+    __syncthreads();
+    if (!sh.flag) return;
+    __threadfence();
+    merge_row<kBf16, kKind>(p, row, canvas, inv_tau, rowp, sh);
+}
+
+}  // namespace
+
+cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s) {
+    const long long grid = static_cast<long long>(p.R) * p.segs;
+    if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const dim3 g(static_cast<unsigned>(grid)), b(kPassThreads);
+#define DG_LAUNCH(BF, K) logits_pass_kernel<BF, K><<<g, b, 0, s>>>(p)
+    if (is_bf16) {
+        if (kind == kPassSampler) DG_LAUNCH(true, kPassSampler);
+        else if (kind == kPassStats) DG_LAUNCH(true, kPassStats);
+        else DG_LAUNCH(true, kPassCE);
+    } else {
+        if (kind == kPassSampler) DG_LAUNCH(false, kPassSampler);
+        else if (kind == kPassStats) DG_LAUNCH(false, kPassStats);
+        else DG_LAUNCH(false, kPassCE);
+    }
+#undef DG_LAUNCH
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace dg

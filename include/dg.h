@@ -1,0 +1,175 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) sampler library for block-parallel
+ * uniform-noise discrete diffusion (DiffusionGemma-style denoising).
+ *
+ * Pages cited: DiffusionGemma Technical Report, hyper.ai paper summary,
+ *   section "Method"  -- forward probability path
+ *       P(X_t = x_t | X_0 = x_0) = prod_i [kappa_t delta(x_t^i, x_0^i) + (1 - kappa_t)/V],
+ *     the schedule kappa (monotone, kappa_0 = 1, kappa_1 = 0), the Step
+ *     reverse transition, the per-iteration update
+ *       p0 = Softmax(L_t / tau_t),  z = FFW(p0 E),  x_{t-dt} ~ Step(x_t, p0),
+ *     and the canvas loss L = -sum_{i=1..C} log p(x_0^i | x_t, z_t, H);
+ *   section "Dataset" -- training sequences of P prompt tokens + K canvases of
+ *     C tokens; the decoder loss on one canvas per sequence chosen uniformly.
+ *
+ * Conventions shared by every entry point
+ *   - Every function returns an int status (dg_status).  On failure nothing
+ *     has been launched, and dg_last_error() (thread-local) says why.
+ *   - Device buffers are owned by the caller and are never freed or kept by
+ *     the library.  The library allocates no device memory: scratch comes
+ *     from a caller workspace sized by the matching *_workspace_size query.
+ *     A workspace must be zero-filled before its first use, and again before
+ *     it is reused for a call of a different shape (rows, V, n_seq): the
+ *     layout inside it depends on the shape.  Every call that returns DG_OK
+ *     leaves the counters inside it at zero, so one workspace serves any
+ *     number of successive same-shape calls on one stream.  Two calls that
+ *     run at the same time need two workspaces.
+ *   - Per-canvas scalars (t, dt, inv_tau) are HOST arrays, read during the
+ *     call; everything else named "device" is device memory.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream).  Arguments are checked before any
+ *     launch; the device work itself reports no errors.
+ *   - Logits rows: element (r, v) lives at logits + r*ld + v (elements), the
+ *     base is 16-byte aligned and ld*sizeof(element) is a multiple of 16.
+ *     Logits must be finite or -inf (a masked token); NaN is not supported.
+ *   - Random numbers: Philox4x32-10 (Salmon et al., SC'11) with key
+ *     (seed & 0xffffffff, seed >> 32); counter word 3 names the use:
+ *       0 token Gumbel     (v >> 2, row, step, 0), word v & 3
+ *       1 Step             (0, row, step, 1): word 0 branch, word 1 token
+ *       2 forward noise    (j, b, 0, 2): word 0 keep, word 1 token
+ *       3 loss canvas      (0, b, 0, 3): word 0
+ *       4 chunk Gumbel     (c >> 2, row, step, 4), word c & 3
+ *     A word w becomes u = (2 (w >> 9) + 1) 2^-24 for a Gumbel variate
+ *     -ln(-ln u), u = w 2^-32 for a comparison with a probability, and
+ *     floor(w n / 2^32) for an index in [0, n).
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dg_stream_t; /* same type as cudaStream_t */
+
+typedef enum dg_status {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = 1, /* a size, enum, pointer or scalar is out of range */
+    DG_ERR_ALIGNMENT = 2,   /* a pointer or leading dimension breaks the 16-byte rule */
+    DG_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query */
+    DG_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
+    DG_ERR_UNSUPPORTED = 5  /* valid request this build does not handle (e.g. no sm_100 device) */
+} dg_status;
+
+typedef enum dg_dtype { DG_F32 = 0, DG_BF16 = 1 } dg_dtype;
+
+/* Noise schedule kappa_t.  The pages fix only kappa_0 = 1, kappa_1 = 0 and
+ * monotone decrease; the forms are: LINEAR 1 - t, COSINE cos^2(pi t / 2). */
+typedef enum dg_schedule { DG_SCHED_LINEAR = 0, DG_SCHED_COSINE = 1 } dg_schedule;
+
+/* How x0_hat is drawn from p0 = softmax(l * inv_tau).
+ * SAMPLE: two-level Gumbel-max.  Level 1 scores each chunk of
+ *   DG_GUMBEL_CHUNK consecutive ids (the last one ragged) with its
+ *   log-sum-exp plus a chunk Gumbel variate; level 2 takes
+ *   argmax_v l'_v + G_v inside the winning chunk.  Ties go to the lowest
+ *   chunk, then the lowest id.  This draws exactly from softmax(l'); with
+ *   V <= DG_GUMBEL_CHUNK it is plain Gumbel-max.
+ * GREEDY: x0_hat = argmax_v l_v (lowest id on ties). */
+typedef enum dg_x0_mode { DG_X0_SAMPLE = 0, DG_X0_GREEDY = 1 } dg_x0_mode;
+
+#define DG_GUMBEL_CHUNK 512
+#define DG_MAX_CANVASES 256 /* canvases (B, n_seq) per call */
+
+/* Human-readable reason for the last failure on this thread ("" if none). */
+const char* dg_last_error(void);
+/* Library version string. */
+const char* dg_version(void);
+/* Number of kernels this library has launched in this process so far. */
+uint64_t dg_launch_count(void);
+
+/* ------------------------------------------------------------------------ */
+/* Sampler step (section "Method": p0 = Softmax(L_t / tau_t) and             */
+/* x_{t-dt} ~ Step(x_t, p0)).  For each row r = b*C + i of B canvases:        */
+/*   lse[r]      = log sum_v exp(l'_v),  l' = logits[r, :V] * inv_tau[b]     */
+/*   max_prob[r] = max_v p0_v,  entropy[r] = -sum_v p0_v ln p0_v             */
+/*   argmax[r]   = argmax_v logits[r, v] (lowest v on ties)                  */
+/*   x0_hat[r]   ~ p0 (mode SAMPLE) or argmax[r] (mode GREEDY)               */
+/*   x_next[r]   ~ P(X_s | X_t = x_t[r], X_0 = x0_hat[r]), s = max(t - dt, 0)*/
+/*                 the exact posterior of the forward path; branch[r] = 0    */
+/*                 stayed at x_t, 1 jumped to x0_hat, 2 drew a uniform token.*/
+/*                 If kappa(s) <= kappa(t) (dt = 0) x_next = x_t, branch 0.  */
+/* logits: device, DG_F32 or DG_BF16, [B*C, ld] (ld >= V).                   */
+/* x_t: device int32 [B*C], ids in [0, V).                                   */
+/* t, dt: host double [B], 0 <= t <= 1, dt >= 0.                             */
+/* inv_tau: host float [B] (> 0, finite) or NULL for 1.                      */
+/* Outputs (device, [B*C]): x_next int32 (required); x0_hat, argmax int32,   */
+/* max_prob, lse, entropy float32, branch uint8 -- each may be NULL.         */
+/* 1 <= B <= DG_MAX_CANVASES, C >= 1, 1 <= V < 2^31, B*C < 2^31.             */
+/* ------------------------------------------------------------------------ */
+size_t dg_sampler_step_workspace_size(int32_t rows, int32_t V);
+
+int dg_sampler_step(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t, int32_t B,
+                    int32_t C, int32_t V, int schedule, const double* t, const double* dt,
+                    const float* inv_tau, uint64_t seed, uint32_t step, int x0_mode,
+                    int32_t* x_next, int32_t* x0_hat, int32_t* argmax, float* max_prob,
+                    float* lse, float* entropy, uint8_t* branch, void* workspace,
+                    size_t workspace_bytes, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Self-conditioning input (section "Method": z = FFW(p0 E)).  The trained   */
+/* FFW is not part of this library; it computes the expected embedding      */
+/*   z[r, :] = sum_v p0[r, v] E[v, :],  p0 = softmax(logits[r, :V] * inv_tau[b])*/
+/* on the tensor cores (bf16 operands, fp32 accumulation), z stored bf16.    */
+/* logits: device DG_F32 or DG_BF16 [B*C, ld].                              */
+/* lse: device float [B*C] = log-sum-exp of logits*inv_tau per row, exactly  */
+/*   as dg_sampler_step writes it; or NULL, in which case the library runs  */
+/*   its own statistics pass first.                                          */
+/* E: device [V, d] row-major, DG_BF16 (DG_F32 is rounded to bf16 into the   */
+/*   workspace first).  d is a multiple of 64, 64 <= d <= 16384.             */
+/* z: device bf16 [B*C, d] row-major.                                        */
+/* ------------------------------------------------------------------------ */
+size_t dg_selfcond_workspace_size(int32_t rows, int32_t V, int32_t d, int logits_dtype,
+                                  int embed_dtype, int have_lse);
+
+int dg_selfcond(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
+                const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d,
+                void* z, void* workspace, size_t workspace_bytes, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Training-side forward corruption (section "Method": forward path, noisy   */
+/* tokens drawn uniformly from the vocabulary; section "Dataset": P + K*C    */
+/* layout, one loss canvas per sequence chosen uniformly).                   */
+/* x0: device int32 [n_seq, P + K*C].  Prompt tokens are copied; each canvas*/
+/* token j of sequence b is kept if w0 2^-32 < kappa(t[b]) and otherwise set*/
+/* to floor(w1 V / 2^32).  canvas_idx[b] = floor(w0' K / 2^32).               */
+/* t: host double [n_seq] in [0, 1].  x_t: device int32 like x0 (may not     */
+/* alias x0).  canvas_idx: device int32 [n_seq] or NULL.  No workspace.      */
+/* ------------------------------------------------------------------------ */
+int dg_forward_noise(const int32_t* x0, int32_t n_seq, int32_t P, int32_t K, int32_t C, int32_t V,
+                     int schedule, const double* t, uint64_t seed, int32_t* x_t,
+                     int32_t* canvas_idx, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Canvas cross-entropy (section "Method": L = -sum_i log p(x_0^i | ...)) on */
+/* the chosen canvas of each sequence (section "Dataset").                   */
+/* logits: device DG_F32 or DG_BF16 [n_seq*C, ld]; row b*C + i predicts      */
+/* target x0[b, P + canvas_idx[b]*C + i].  Outputs (device float):           */
+/*   loss_rows [n_seq*C] = lse - logit[target], lse_rows [n_seq*C] (may be   */
+/*   NULL), loss_seq [n_seq] = sum over the C rows (may be NULL).            */
+/* canvas_idx: device int32 [n_seq], values in [0, K).                       */
+/* ------------------------------------------------------------------------ */
+size_t dg_canvas_ce_workspace_size(int32_t n_seq, int32_t C, int32_t V);
+
+int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t* x0,
+                 const int32_t* canvas_idx, int32_t n_seq, int32_t P, int32_t K, int32_t C,
+                 int32_t V, float* loss_rows, float* loss_seq, float* lse_rows, void* workspace,
+                 size_t workspace_bytes, dg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

@@ -22,7 +22,7 @@ _SRC = os.path.join(_HERE, "dg_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libdg_oracle.so")
 
 # Chunk width of the two-level Gumbel-max draw (level 1 scores chunks of Q ids).
-GUMBEL_CHUNK = 2048
+GUMBEL_CHUNK = 512
 
 
 def build(force: bool = False) -> str:

@@ -1,0 +1,128 @@
+"""CPU checks of the C ABI: the library builds for sm_100a, loads, exports every function
+include/dg.h declares, and rejects bad arguments with a status and a message before any
+launch (these calls never reach a device, so they are safe with or without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import discrete_diffusion_lm_b200 as dg
+from discrete_diffusion_lm_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+FAKE = 1 << 20  # an aligned non-null address that is never dereferenced (calls fail validation first)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return dg.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"dg_sampler_step", "dg_selfcond", "dg_forward_noise", "dg_canvas_ce"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in dg.h but not exported"
+
+
+def test_version_and_launch_count(L):
+    assert dg.dg_version().startswith("dg ")
+    assert dg.dg_launch_count() >= 0
+
+
+def _step(L, **kw):
+    a = dict(logits=FAKE, dtype=1, ld=1024, x_t=FAKE, B=1, C=16, V=1024, sched=0, t=[0.5], dt=[0.1],
+             inv_tau=None, seed=0, step=0, mode=0, x_next=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    B = a["B"]
+    t = (ctypes.c_double * max(B, 1))(*(a["t"] * max(B, 1))[:max(B, 1)]) if a["t"] is not None else None
+    dt = (ctypes.c_double * max(B, 1))(*(a["dt"] * max(B, 1))[:max(B, 1)]) if a["dt"] is not None else None
+    it = None if a["inv_tau"] is None else (ctypes.c_float * max(B, 1))(*([a["inv_tau"]] * max(B, 1)))
+    rc = L.dg_sampler_step(a["logits"], a["dtype"], a["ld"], a["x_t"], B, a["C"], a["V"], a["sched"], t, dt, it,
+                           ctypes.c_uint64(a["seed"]), ctypes.c_uint32(a["step"]), a["mode"], a["x_next"], None,
+                           None, None, None, None, None, a["ws"], a["ws_bytes"], None)
+    return rc, dg.dg_last_error()
+
+
+@pytest.mark.parametrize("kw,code,frag", [
+    (dict(logits=None), 1, "logits is NULL"),
+    (dict(dtype=7), 1, "dtype"),
+    (dict(V=0), 1, "V = 0"),
+    (dict(ld=1000), 1, "smaller than V"),
+    (dict(logits=FAKE + 2), 2, "16-byte"),
+    (dict(ld=1028, V=1025), 2, "multiple of 16"),
+    (dict(B=0), 1, "B = 0"),
+    (dict(B=300), 1, "B = 300"),
+    (dict(C=0), 1, "C = 0"),
+    (dict(x_next=None), 1, "required"),
+    (dict(t=None), 1, "required"),
+    (dict(sched=5), 1, "schedule"),
+    (dict(mode=3), 1, "x0_mode"),
+    (dict(ws=None), 3, "workspace"),
+    (dict(ws_bytes=16), 3, "workspace"),
+    (dict(t=[1.5]), 1, "outside [0, 1]"),
+    (dict(t=[float("nan")]), 1, "outside [0, 1]"),
+    (dict(dt=[-0.1]), 1, "dt[0]"),
+    (dict(inv_tau=0.0), 1, "inv_tau"),
+    (dict(inv_tau=float("inf")), 1, "inv_tau"),
+])
+def test_sampler_step_rejects(L, kw, code, frag):
+    rc, msg = _step(L, **kw)
+    assert rc == code, msg
+    assert frag in msg
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_cuda_error(L):
+    rc, msg = _step(L)
+    assert rc in (4, 5), msg  # DG_ERR_CUDA (no device) or DG_ERR_UNSUPPORTED
+    assert msg
+
+
+def test_forward_noise_rejects(L):
+    t = (ctypes.c_double * 2)(0.5, 0.5)
+    f = L.dg_forward_noise
+    assert f(FAKE, 0, 0, 1, 4, 10, 1, t, 0, FAKE + 64, None, None) == 1      # n_seq = 0
+    assert f(FAKE, 2, -1, 1, 4, 10, 1, t, 0, FAKE + 64, None, None) == 1     # P < 0
+    assert f(FAKE, 2, 0, 1, 4, 10, 7, t, 0, FAKE + 64, None, None) == 1      # schedule
+    assert f(FAKE, 2, 0, 1, 4, 10, 1, t, 0, None, None, None) == 1           # x_t missing
+    assert f(FAKE, 2, 0, 1, 4, 10, 1, t, 0, FAKE, None, None) == 1           # x_t aliases x0
+    bad_t = (ctypes.c_double * 2)(0.5, 2.0)
+    assert f(FAKE, 2, 0, 1, 4, 10, 1, bad_t, 0, FAKE + 64, None, None) == 1  # t outside [0, 1]
+    assert "t[1]" in dg.dg_last_error()
+
+
+def test_selfcond_rejects(L):
+    it = None
+    f = L.dg_selfcond
+    assert f(FAKE, 1, 1024, 1, 16, 1024, it, None, FAKE, 1, 100, FAKE, FAKE, 1 << 30, None) == 1  # d % 64
+    assert f(FAKE, 1, 1024, 1, 16, 1024, it, None, None, 1, 64, FAKE, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, 1, 1024, 1, 16, 1024, it, None, FAKE + 8, 1, 64, FAKE, FAKE, 1 << 30, None) == 2
+    assert f(FAKE, 1, 1024, 1, 16, 1024, it, None, FAKE, 1, 64, FAKE, FAKE, 8, None) == 3
+    assert f(FAKE, 1, 1024, 1, 16, 1024, it, None, FAKE, 9, 64, FAKE, FAKE, 1 << 30, None) == 1
+
+
+def test_canvas_ce_rejects(L):
+    f = L.dg_canvas_ce
+    assert f(FAKE, 1, 1024, FAKE, FAKE, 2, 4, 2, 8, 1024, None, None, None, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, 1, 1024, FAKE, FAKE, 2, 4, 0, 8, 1024, FAKE, None, None, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, 1, 1024, FAKE, FAKE, 2, 4, 2, 8, 1024, FAKE, None, None, FAKE, 4, None) == 3
+
+
+def test_workspace_queries(L):
+    assert dg.dg_sampler_step_workspace_size(256, 262144) >= 256 * 128 * 16
+    assert dg.dg_sampler_step_workspace_size(0, 5) == 0
+    assert dg.dg_canvas_ce_workspace_size(8, 256, 262144) >= 2048 * 128 * 16
+    assert dg.dg_selfcond_workspace_size(256, 262144, 2048, 1, 1, True) >= 0
+    assert dg.dg_selfcond_workspace_size(256, 262144, 2048, 1, 0, True) >= 262144 * 2048 * 2
