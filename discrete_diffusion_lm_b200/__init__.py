@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.dg_last_error.restype = ctypes.c_char_p
         L.dg_version.restype = ctypes.c_char_p
         L.dg_launch_count.restype = _u64
+        L.dg_device_error.argtypes = [_p]
         L.dg_sampler_step_workspace_size.argtypes = [_i32, _i32]
         L.dg_sampler_step_workspace_size.restype = _sz
         L.dg_sampler_step.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32, _int,
@@ -75,6 +76,14 @@ def dg_version() -> str:
 
 def dg_launch_count() -> int:
     return int(lib().dg_launch_count())
+
+
+def dg_device_error() -> int:
+    """Synchronize the device and return (and clear) the library's device error word:
+    0 = no kernel reported a problem, 1 = a kernel gave up on a bounded wait."""
+    code = ctypes.c_int(0)
+    _check("dg_device_error", lib().dg_device_error(ctypes.byref(code)))
+    return code.value
 
 
 def _check(fn: str, rc: int):

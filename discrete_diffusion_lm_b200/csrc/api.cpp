@@ -172,6 +172,18 @@ const char* dg_version(void) { return "dg 0.1 (sm_100a)"; }
 
 uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int dg_device_error(int* code) {
+    g_last_error.clear();
+    if (!code) return fail(DG_ERR_INVALID_ARG, "code is NULL");
+    int rc;
+    if ((rc = check_device()) != DG_OK) return rc;
+    const cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    const cudaError_t r = read_and_clear_device_error(code);
+    if (r != cudaSuccess) return cuda_fail(r, "reading the device error word");
+    return DG_OK;
+}
+
 size_t dg_sampler_step_workspace_size(int32_t rows, int32_t V) {
     if (rows < 1 || V < 1) return 0;
     return pass_ws_bytes(rows, V, 0);

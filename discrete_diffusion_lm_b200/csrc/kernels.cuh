@@ -77,16 +77,16 @@ struct SelfcondParams {
     const float* lse;    // [R]
     const uint16_t* E;   // bf16 [V, d]
     uint16_t* z;         // bf16 [R, d]
-    float* partial;      // fp32 [splits, R, d] (when splits > 1)
-    uint32_t* tile_ticket;
+    float* partial;      // fp32 [splits, R, d] (when the vocabulary is split)
     int32_t R, C, V, d;
-    int32_t splits;
     float inv_tau[DG_MAX_CANVASES];
 };
 
 size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d);
 cudaError_t launch_selfcond(const SelfcondParams& p, cudaStream_t s);
 cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s);
+// Reads (synchronously) and clears the error word set by a kernel whose bounded wait expired.
+cudaError_t read_and_clear_device_error(int* out);
 
 // Count of kernels launched by the library (for the launch-count query).
 void note_launches(uint64_t n);

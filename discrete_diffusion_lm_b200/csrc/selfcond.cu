@@ -1,22 +1,552 @@
-// placeholder: replaced by the tcgen05 contraction
+// Self-conditioning contraction z = softmax(l * inv_tau) E on the sm_100a tensor cores.
+//
+// DiffusionGemma Technical Report (hyper.ai summary), section "Method": the update
+// z_{t-dt} = FFW(p0 E) with p0 = Softmax(L_t / tau_t) and E the token-embedding matrix.  The
+// expected embedding p0 E is the dense contraction computed here (the trained FFW is not).
+//
+// One CTA computes a 128-row x kNT-column tile of z over a contiguous range of the vocabulary
+// (split-K).  Per stage of kKBlock = 32 ids:
+//   * a producer thread TMA-loads the E tile [32 ids x kNT] (MN-major, 128-byte swizzle, boxes of
+//     64 columns) and the logits tile [128 rows x 32 ids] (64-byte swizzle for bf16);
+//   * four softmax warps turn each thread's logits row into p = exp2(l * a - lse * log2 e), i.e.
+//     softmax(l') with the row's log-sum-exp from the logits pass, round it to bf16 and write it
+//     back in the K-major 64-byte-swizzled layout the tensor core reads as operand A;
+//   * one thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into a TMEM accumulator of
+//     128 lanes x kNT columns and commits the stage back to the producer.
+// Because lse is known, p is final when it is formed: no running-max rescale of the accumulator is
+// needed.  After the last stage the softmax warps read the accumulator out of TMEM (tcgen05.ld)
+// and store bf16 z, or fp32 partial sums that a second kernel adds in a fixed order.
+// Every mbarrier wait is bounded: on expiry the CTA records an error, stops issuing work, waits
+// (bounded) for its in-flight copies and frees its TMEM.
+#include <cuda.h>  // CUtensorMap and its enums (the encoder itself is fetched from the driver at run time)
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
+
 namespace dg {
+
+__device__ int g_device_error = 0;  // set by a kernel whose bounded wait expired
+
 namespace {
-__global__ void convert_f32_bf16_kernel(const float* in, uint16_t* out, int64_t n) {
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i < n) {
+
+constexpr int kKBlock = 32;  // vocabulary ids per pipeline stage
+constexpr int kTileM = 128;  // rows per CTA = TMEM lanes
+constexpr int kNumSoftmaxWarps = 4;
+constexpr int kThreads = 64 + 32 * kNumSoftmaxWarps;  // producer warp, MMA warp, softmax warps
+constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at the boost clock
+
+struct alignas(64) KernelParams {
+    CUtensorMap tm_logits;  // [R, V], box 128 rows x (64 bytes of ids)
+    CUtensorMap tm_E;       // [V, d], box 32 ids x 64 columns
+    const float* lse;
+    uint16_t* z;
+    float* partial;
+    int32_t R, C, V, d;
+    int32_t n_tiles, splits, total_kb;
+    float inv_tau[DG_MAX_CANVASES];
+};
+
+template <bool kBf16, int kNT>
+struct Cfg {
+    static constexpr uint32_t kEBytes = kNT * kKBlock * 2;
+    static constexpr uint32_t kLBytes = kTileM * kKBlock * (kBf16 ? 2 : 4);
+    static constexpr uint32_t kPBytes = kBf16 ? 0 : kTileM * kKBlock * 2;  // bf16 writes p in place
+    static constexpr uint32_t kStageBytes = kEBytes + kLBytes + kPBytes;
+    static constexpr int kStagesFit = static_cast<int>((200u * 1024u) / kStageBytes);
+    static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
+    static constexpr uint32_t kBarrierBytes = 256;
+    static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+    static_assert(kStages >= 2, "pipeline needs two stages");
+    static_assert(kEBytes % 1024 == 0 && kLBytes % 1024 == 0 && kPBytes % 1024 == 0, "1 KB-aligned stage parts");
+};
+
+// ------------------------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity to complete.  Gives up (returning false) when another
+// thread of the CTA has aborted or after kWaitLimitCycles, recording the expiry.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_device_error, 1);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int32_t c0, int32_t c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tcgen05_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tcgen05_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// UMMA shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
+// units), descriptor version 1 (sm_100), swizzle mode in bits 61..63 (2 = 128 B, 4 = 64 B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
+    uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
+    return d;
+}
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+
+// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, A K-major, B MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// p for 8 consecutive bf16 logits held in one 16-byte chunk, packed back as 8 bf16.
+__device__ __forceinline__ uint4 softmax_chunk_bf16(uint4 c, float a, float nb) {
+    uint4 o;
+    o.x = pack_bf16x2(ex2_approx(fmaf(bf16_lo(c.x), a, nb)), ex2_approx(fmaf(bf16_hi(c.x), a, nb)));
+    o.y = pack_bf16x2(ex2_approx(fmaf(bf16_lo(c.y), a, nb)), ex2_approx(fmaf(bf16_hi(c.y), a, nb)));
+    o.z = pack_bf16x2(ex2_approx(fmaf(bf16_lo(c.z), a, nb)), ex2_approx(fmaf(bf16_hi(c.z), a, nb)));
+    o.w = pack_bf16x2(ex2_approx(fmaf(bf16_lo(c.w), a, nb)), ex2_approx(fmaf(bf16_hi(c.w), a, nb)));
+    return o;
+}
+__device__ __forceinline__ uint32_t softmax_pair_f32(uint32_t x, uint32_t y, float a, float nb) {
+    return pack_bf16x2(ex2_approx(fmaf(__uint_as_float(x), a, nb)), ex2_approx(fmaf(__uint_as_float(y), a, nb)));
+}
+
+template <bool kBf16, int kNT>
+__global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_constant__ KernelParams p) {
+    using G = Cfg<kBf16, kNT>;
+    constexpr int kStages = G::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* efull = reinterpret_cast<uint64_t*>(smem + kStages * G::kStageBytes);
+    uint64_t* lfull = efull + kStages;
+    uint64_t* pready = lfull + kStages;
+    uint64_t* empty = pready + kStages;
+    uint64_t* accum = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    int bid = blockIdx.x;
+    const int split = bid % p.splits;
+    bid /= p.splits;
+    const int nt = bid % p.n_tiles;
+    const int mt = bid / p.n_tiles;
+    const int kb0 = static_cast<int>(static_cast<long long>(split) * p.total_kb / p.splits);
+    const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.total_kb / p.splits);
+    const int nkb = kb1 - kb0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&efull[s], 1);
+            mbar_init(&lfull[s], 1);
+            mbar_init(&pready[s], 32 * kNumSoftmaxWarps);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accum, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(static_cast<uint32_t>(kNT))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tcgen05_before_sync();
+    __syncthreads();
+    tcgen05_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
+                uint8_t* st = smem + s * G::kStageBytes;
+                const int32_t k0 = (kb0 + i) * kKBlock;
+                mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
+                tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mt * kTileM, &lfull[s]);
+                mbar_arrive_expect_tx(&efull[s], G::kEBytes);
+#pragma unroll
+                for (int b = 0; b < kNT / 64; ++b)
+                    tma_load_2d(st + b * (64 * kKBlock * 2), &p.tm_E, nt * kNT + 64 * b, k0, &efull[s]);
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                // let the copies already issued land before the CTA's shared memory goes away
+                for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i) {
+                    const int s = i % kStages;
+                    const uint32_t ph = (i / kStages) & 1;
+                    const long long t0 = clock64();
+                    while (!(mbar_try_wait(&lfull[s], ph) && mbar_try_wait(&efull[s], ph)) &&
+                           clock64() - t0 < kWaitLimitCycles) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr int kMmaN = kNT > 256 ? 256 : kNT;
+            constexpr uint32_t idesc = idesc_bf16(kTileM, kMmaN);
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&efull[s], ph, abort_flag)) break;
+                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                tcgen05_after_sync();
+                uint8_t* st = smem + s * G::kStageBytes;
+                const uint32_t a_base = smem_u32(st + G::kEBytes + (kBf16 ? 0 : G::kLBytes));
+                const uint32_t b_base = smem_u32(st);
+#pragma unroll
+                for (int ks = 0; ks < kKBlock / 16; ++ks) {
+                    // A: 128 rows x 16 ids, K-major, rows of 64 bytes, 8-row atoms of 512 bytes
+                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 512, kLayoutSw64);
+#pragma unroll
+                    for (int nh = 0; nh < kNT / kMmaN; ++nh) {
+                        // B: 16 ids x kMmaN columns, MN-major, 64-column boxes 4 KB apart, 8-id atoms of 1 KB
+                        const uint64_t bdesc =
+                            smem_desc(b_base + nh * (kMmaN / 64) * (64 * kKBlock * 2) + ks * 2048, 64 * kKBlock * 2,
+                                      1024, kLayoutSw128);
+                        umma_bf16(tmem + nh * kMmaN, adesc, bdesc, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&empty[s]);
+            }
+            umma_commit(accum);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax + epilogue
+        const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ..
+        const int row = quarter * 32 + lane;
+        const int32_t r = mt * kTileM + row;
+        const bool valid = r < p.R;
+        const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
+        const float a = it * kLog2e;
+        const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
+        for (int i = 0; i < nkb; ++i) {
+            const int s = i % kStages;
+            const uint32_t ph = (i / kStages) & 1;
+            if (!mbar_wait(&lfull[s], ph, abort_flag)) break;
+            uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
+            if (kBf16) {
+                // row of 32 bf16 = 64 bytes; 16-byte chunk j stored at j ^ ((row >> 1) & 3)
+                uint8_t* rb = lt + row * 64;
+                const int sw = (row >> 1) & 3;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4* q = reinterpret_cast<uint4*>(rb + ((j ^ sw) << 4));
+                    *q = softmax_chunk_bf16(*q, a, nb);
+                }
+            } else {
+                // fp32 row of 32 ids = 128 bytes, chunk j at j ^ (row & 7); p goes to the bf16 tile
+                const uint8_t* rb = lt + row * 128;
+                uint8_t* pb = lt + G::kLBytes + row * 64;
+                const int sw8 = row & 7, sw4 = (row >> 1) & 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 c0 = *reinterpret_cast<const uint4*>(rb + (((2 * q) ^ sw8) << 4));
+                    const uint4 c1 = *reinterpret_cast<const uint4*>(rb + (((2 * q + 1) ^ sw8) << 4));
+                    uint4 o;
+                    o.x = softmax_pair_f32(c0.x, c0.y, a, nb);
+                    o.y = softmax_pair_f32(c0.z, c0.w, a, nb);
+                    o.z = softmax_pair_f32(c1.x, c1.y, a, nb);
+                    o.w = softmax_pair_f32(c1.z, c1.w, a, nb);
+                    *reinterpret_cast<uint4*>(pb + ((q ^ sw4) << 4)) = o;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&pready[s]);
+        }
+        if (mbar_wait(accum, 0, abort_flag)) {
+            tcgen05_after_sync();
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            for (int c = 0; c < kNT; c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(lane_base + c, v);
+                if (valid) {
+                    const int32_t col = nt * kNT + c;
+                    if (p.splits == 1) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.z + static_cast<size_t>(r) * p.d + col);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                            dst[q] = o;
+                        }
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.partial + (static_cast<size_t>(split) * p.R + r) * p.d + col);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    tcgen05_before_sync();
+    __syncthreads();
+    tcgen05_after_sync();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(static_cast<uint32_t>(kNT))
+                     : "memory");
+}
+
+// z[i] = bf16(sum_s partial[s][i]) in a fixed order (deterministic).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ partial, uint2* __restrict__ z,
+                                                            int64_t n4, int splits) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float4 acc = __ldcs(partial + i);
+        for (int s = 1; s < splits; ++s) {
+            const float4 v = __ldcs(partial + static_cast<int64_t>(s) * n4 + i);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        z[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
+}
+
+__global__ void convert_f32_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const __nv_bfloat16 h = __float2bfloat16_rn(in[i]);
         out[i] = *reinterpret_cast<const uint16_t*>(&h);
     }
 }
+
+// ------------------------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+cudaError_t encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int pick_ntile(int d) { return d % 512 == 0 ? 512 : d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64; }
+
+int num_sms() {
+    static std::atomic<int> cached{0};
+    int v = cached.load();
+    if (v == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cached.store(v);
+    }
+    return v;
+}
+
+// Split the vocabulary so that the grid is about one wave of CTAs (one CTA per SM).
+void plan(int R, int V, int d, int* m_tiles, int* n_tiles, int* splits, int* total_kb) {
+    *m_tiles = (R + kTileM - 1) / kTileM;
+    *n_tiles = d / pick_ntile(d);
+    *total_kb = (V + kKBlock - 1) / kKBlock;
+    const int tiles = *m_tiles * *n_tiles;
+    int s = num_sms() / tiles;
+    if (s < 1) s = 1;
+    if (s > *total_kb) s = *total_kb;
+    *splits = s;
+}
+
+template <bool kBf16, int kNT>
+cudaError_t launch_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
+    using G = Cfg<kBf16, kNT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(selfcond_kernel<kBf16, kNT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(G::kSmemBytes));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    selfcond_kernel<kBf16, kNT><<<grid, kThreads, G::kSmemBytes, st>>>(kp);
+    return cudaGetLastError();
+}
+
 }  // namespace
-size_t selfcond_partial_bytes(int32_t, int32_t, int32_t) { return 0; }
-cudaError_t launch_selfcond(const SelfcondParams&, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s) {
-    const int64_t blocks = (n + 255) / 256;
-    convert_f32_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(in, out, n);
+
+size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d) {
+    int mt, ntl, s, tkb;
+    if (R < 1 || V < 1 || d < 64) return 0;
+    plan(R, V, d, &mt, &ntl, &s, &tkb);
+    return s > 1 ? static_cast<size_t>(s) * R * d * sizeof(float) : 0;
+}
+
+cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
+    static thread_local KernelParams kp;
+    std::memset(&kp, 0, sizeof(kp));
+    int m_tiles, n_tiles, splits, total_kb;
+    plan(sp.R, sp.V, sp.d, &m_tiles, &n_tiles, &splits, &total_kb);
+    const int nt = pick_ntile(sp.d);
+    cudaError_t e;
+    if (sp.logits_bf16)
+        e = encode_2d(&kp.tm_logits, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.logits, sp.V, sp.R,
+                      static_cast<uint64_t>(sp.ld) * 2, kKBlock, kTileM, CU_TENSOR_MAP_SWIZZLE_64B);
+    else
+        e = encode_2d(&kp.tm_logits, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.logits, sp.V, sp.R,
+                      static_cast<uint64_t>(sp.ld) * 4, kKBlock, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = encode_2d(&kp.tm_E, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.E, sp.d, sp.V, static_cast<uint64_t>(sp.d) * 2, 64,
+                  kKBlock, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    kp.lse = sp.lse;
+    kp.z = sp.z;
+    kp.partial = sp.partial;
+    kp.R = sp.R;
+    kp.C = sp.C;
+    kp.V = sp.V;
+    kp.d = sp.d;
+    kp.n_tiles = n_tiles;
+    kp.splits = splits;
+    kp.total_kb = total_kb;
+    std::memcpy(kp.inv_tau, sp.inv_tau, sizeof(kp.inv_tau));
+    const int grid = m_tiles * n_tiles * splits;
+#define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st)
+    if (sp.logits_bf16) {
+        if (nt == 512) DG_SC(true, 512);
+        else if (nt == 256) DG_SC(true, 256);
+        else if (nt == 128) DG_SC(true, 128);
+        else DG_SC(true, 64);
+    } else {
+        if (nt == 512) DG_SC(false, 512);
+        else if (nt == 256) DG_SC(false, 256);
+        else if (nt == 128) DG_SC(false, 128);
+        else DG_SC(false, 64);
+    }
+#undef DG_SC
+    note_launches(1);
+    if (e != cudaSuccess || splits == 1) return e;
+    const int64_t n4 = static_cast<int64_t>(sp.R) * sp.d / 4;
+    const int blocks = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, 4LL * num_sms()));
+    splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(sp.partial),
+                                                reinterpret_cast<uint2*>(sp.z), n4, splits);
     note_launches(1);
     return cudaGetLastError();
 }
+
+cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s) {
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 8LL * num_sms()));
+    convert_f32_bf16_kernel<<<blocks, 256, 0, s>>>(in, out, n);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(int* out) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    }
+    *out = v;
+    return e;
+}
+
 }  // namespace dg

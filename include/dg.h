@@ -89,6 +89,12 @@ const char* dg_last_error(void);
 const char* dg_version(void);
 /* Number of kernels this library has launched in this process so far. */
 uint64_t dg_launch_count(void);
+/* Synchronizes the current device, then stores in *code (and clears) the
+ * library's device error word: 0 if no kernel has reported a problem, 1 if a
+ * kernel gave up on a bounded wait (its outputs are then incomplete).  Every
+ * wait inside the library's kernels is bounded (about two seconds), so a
+ * stalled pipeline ends with this code instead of hanging the device. */
+int dg_device_error(int* code);
 
 /* ------------------------------------------------------------------------ */
 /* Sampler step (section "Method": p0 = Softmax(L_t / tau_t) and             */

@@ -1,0 +1,133 @@
+"""GPU-vs-oracle parity of the self-conditioning contraction z = softmax(l * inv_tau) E
+(tcgen05 tensor cores) through the C ABI.
+
+Bar: relative Frobenius error <= 2e-2 against the oracle's double-precision z, on every row
+for the tiny workload and on sampled rows (spanning every M tile) for the larger ones.  At
+full size a property that holds for any size is checked on every row as well: with a column
+of ones in E, that column of z is sum_v p_v = 1 (up to bf16 rounding).
+"""
+import numpy as np
+import pytest
+import torch
+
+import discrete_diffusion_lm_b200 as dg
+from discrete_diffusion_lm_b200 import dg_sampler_step, dg_selfcond, workloads as W
+from oracle import oracle as O
+from tests.parity import Z_REL_FRO, host_f32, rel_fro
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _z_ref(logits, E, rows, inv_tau_rows=None):
+    return O.selfcond_rows(host_f32(logits), host_f32(E), rows, inv_tau_rows)
+
+
+def _device_error_clear():
+    return dg.dg_device_error()
+
+
+@pytest.mark.parametrize("with_lse", [True, False])
+def test_tiny_all_rows(with_lse):
+    cfg = W.TINY
+    logits = W.make_logits(cfg, DEV)
+    E = W.make_embedding(cfg, DEV)
+    lse = None
+    if with_lse:
+        x_t = W.make_canvas(cfg, DEV)
+        lse = dg_sampler_step(logits, x_t, cfg.C, 1.0, 0.125, schedule=cfg.schedule)["lse"]
+    z = dg_selfcond(logits, E, cfg.C, lse=lse)
+    torch.cuda.synchronize()
+    assert _device_error_clear() == 0
+    err = rel_fro(z.float().cpu().numpy(), _z_ref(logits, E, range(cfg.R)))
+    assert err <= Z_REL_FRO, err
+
+
+def test_mid_rows():
+    cfg = W.MID
+    logits = W.make_logits(cfg, DEV)
+    E = W.make_embedding(cfg, DEV)
+    z = dg_selfcond(logits, E, cfg.C)
+    torch.cuda.synchronize()
+    assert _device_error_clear() == 0
+    rows = list(range(0, cfg.R, 7)) + [cfg.R - 1]
+    err = rel_fro(z.float().cpu().numpy()[rows], _z_ref(logits, E, rows))
+    assert err <= Z_REL_FRO, err
+    z2 = dg_selfcond(logits, E, cfg.C)
+    assert torch.equal(z, z2)  # deterministic (fixed-order split-K reduction)
+
+
+def _ones_column_check(logits, E, C, lse, col=5):
+    E1 = E.clone()
+    E1[:, col] = 1.0
+    z = dg_selfcond(logits, E1, C, lse=lse)
+    torch.cuda.synchronize()
+    zc = z[:, col].float()
+    # sum_v p_v = 1: bf16 operands (p rounded to bf16) and a bf16 result keep it within 1e-2
+    assert torch.all((zc - 1.0).abs() < 1e-2), float((zc - 1.0).abs().max())
+
+
+def test_full_vocab_sampled_rows_and_mass():
+    cfg = W.FULL
+    logits = W.make_logits(cfg, DEV)
+    E = W.make_embedding(cfg, DEV)
+    x_t = W.make_canvas(cfg, DEV)
+    lse = dg_sampler_step(logits, x_t, cfg.C, 1.0, 1 / 12, schedule=cfg.schedule)["lse"]
+    z = dg_selfcond(logits, E, cfg.C, lse=lse)
+    torch.cuda.synchronize()
+    assert _device_error_clear() == 0
+    rows = [0, 77, 127, 128, 200, 255]
+    err = rel_fro(z.float().cpu().numpy()[rows], _z_ref(logits, E, rows))
+    assert err <= Z_REL_FRO, err
+    _ones_column_check(logits, E, cfg.C, lse)
+
+
+def test_batched_sampled_rows_and_mass():
+    cfg = W.BATCHED
+    logits = W.make_logits(cfg, DEV)
+    E = W.make_embedding(cfg, DEV)
+    z = dg_selfcond(logits, E, cfg.C)
+    torch.cuda.synchronize()
+    assert _device_error_clear() == 0
+    rows = [0, 1000, 2049, 4095]
+    err = rel_fro(z.float().cpu().numpy()[rows], _z_ref(logits, E, rows))
+    assert err <= Z_REL_FRO, err
+    _ones_column_check(logits, E, cfg.C, None)
+
+
+@pytest.mark.parametrize("R,C,V,ld,d,ldt,edt", [
+    (200, 100, 5000, 5008, 64, torch.bfloat16, torch.bfloat16),
+    (130, 13, 4099, 4104, 128, torch.float32, torch.bfloat16),
+    (64, 64, 777, 784, 256, torch.bfloat16, torch.float32),
+    (129, 43, 3000, 3000, 1536, torch.bfloat16, torch.bfloat16),
+    (1, 1, 33, 40, 512, torch.float32, torch.float32),
+])
+def test_edge_shapes(R, C, V, ld, d, ldt, edt):
+    g = torch.Generator(device=DEV).manual_seed(R + V + d)
+    full = torch.zeros((R, ld), device=DEV, dtype=torch.float32)
+    full[:, :V] = torch.randn((R, V), device=DEV, generator=g) * 2
+    full[0, 3] = 12.0
+    logits = full.to(ldt)
+    E = (torch.randn((V, d), device=DEV, generator=g) * 0.02).to(edt)
+    B = R // C
+    inv_tau = [1.0 + 0.5 * (b % 3) for b in range(B)]
+    z = dg_selfcond(logits, E, C, V=V, inv_tau=inv_tau)
+    torch.cuda.synchronize()
+    assert _device_error_clear() == 0
+    rows = sorted({0, R // 2, R - 1, min(R - 1, 127), min(R - 1, 128)})
+    it_rows = np.array([inv_tau[r // C] for r in range(R)], dtype=np.float32)
+    zr = O.selfcond_rows(host_f32(logits)[:, :ld], host_f32(E), rows, it_rows)
+    err = rel_fro(z.float().cpu().numpy()[rows], zr)
+    assert err <= Z_REL_FRO, err
+
+
+def test_one_hot_rows_pick_embedding_rows():
+    V, d, R = 4096, 256, 128
+    g = torch.Generator(device=DEV).manual_seed(3)
+    E = (torch.randn((V, d), device=DEV, generator=g) * 0.5).to(torch.bfloat16)
+    ids = torch.randint(0, V, (R,), device=DEV, generator=g)
+    logits = torch.full((R, V), -40.0, device=DEV)
+    logits[torch.arange(R, device=DEV), ids] = 40.0
+    z = dg_selfcond(logits.to(torch.bfloat16), E, R)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(z.float(), E[ids].float(), atol=1e-2, rtol=1e-2)
