@@ -1,0 +1,499 @@
+"""Benchmark of the per-step sampler hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one sampler step of the full-vocabulary workload (one canvas of C = 256 tokens,
+V = 262144, d = 2048, bf16 logits and embeddings, cosine schedule, 12 denoising steps per
+block): the logits pass (softmax statistics, argmax, two-level Gumbel-max draw of x0_hat,
+Step posterior) followed by the self-conditioning contraction z = softmax(L) E.  The metric
+is sampler steps/s (and canvas tokens/s = 256 x steps/s), whole job over N GPUs.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier + synchronize on
+both sides, on the device with CUDA events, max over ranks.  Each step reads its own logits
+buffer out of a rotation whose total size is well above the 126 MB L2 (inputs larger than
+L2).  The per-step launches are replayed from CUDA graphs captured once.  N > 1 runs
+independent replicas, one per GPU (the path has no data exchange): weak scaling.
+
+Also reported: the dominant kernel's roofline (measured peaks), an end-to-end figure
+through the public API with host buffers (host->device logits copy and device->host read
+of x_next and z inside the timed region), the training-side kernels (forward noise and
+canvas cross-entropy on the training workload), the CPU oracle timed on a bounded sample
+(rank 0, N = 1), SM clocks sampled during the timed region, and the number of library
+kernel launches in the timed region.
+
+--impl reference times the CPU oracle (the plain C reference of the same computation) on a
+bounded sample of the same workload, on the host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 2**20
+METRIC = "sampler steps/s and canvas tokens/s at C=256,V=262144,d=2048; % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = str(gpu_index)
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.gpu = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        time.sleep(0.25)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ roofline helpers
+def traffic_from_profiles(kernel_file: str, summary_name: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    src = os.path.join(ROOT, "discrete_diffusion_lm_b200", "csrc", kernel_file)
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m_hash = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != digest:
+        return None
+    return int(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    import torch
+    import discrete_diffusion_lm_b200 as dg
+    from discrete_diffusion_lm_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = W.FULL
+    peaks = load_peaks()
+
+    # inputs resident in HBM: a rotation of identical-content logits buffers (> 3x L2 in total)
+    base = W.make_logits(cfg, dev)
+    lbytes = base.numel() * base.element_size()
+    nbuf = max(2, math.ceil(3 * L2_BYTES / lbytes) + 1)
+    bufs = [base] + [base.clone() for _ in range(nbuf - 1)]
+    E = W.make_embedding(cfg, dev)
+    x_buf = [W.make_canvas(cfg, dev), torch.empty(cfg.R, dtype=torch.int32, device=dev)]
+    outs = [{k: torch.empty(cfg.R, dtype=dt, device=dev) for k, dt in
+             (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32), ("max_prob", torch.float32),
+              ("lse", torch.float32), ("entropy", torch.float32), ("branch", torch.uint8))} for _ in range(2)]
+    z = torch.empty((cfg.R, cfg.d), dtype=torch.bfloat16, device=dev)
+    ws_s = torch.zeros(dg.dg_sampler_step_workspace_size(cfg.R, cfg.V), dtype=torch.uint8, device=dev)
+    ws_z = torch.zeros(max(256, dg.dg_selfcond_workspace_size(cfg.R, cfg.V, cfg.d, 1, 1, True)), dtype=torch.uint8,
+                       device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def k1(k):
+        t, dt = cfg.times(k % cfg.steps)
+        o = outs[k % 2]
+        o["x_next"] = x_buf[(k + 1) % 2]
+        dg.dg_sampler_step(bufs[k % nbuf], x_buf[k % 2], cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=k,
+                           out=o, ws=ws_s, stream=stream)
+
+    def k2(k):
+        dg.dg_selfcond(bufs[k % nbuf], E, cfg.C, lse=outs[k % 2]["lse"], z=z, ws=ws_z, stream=stream)
+
+    # one graph per kernel per step of a rotation period (step index and buffer are baked in)
+    period = math.lcm(nbuf, 2 * cfg.steps)
+    with torch.cuda.stream(stream):
+        for k in range(2):
+            k1(k)
+            k2(k)
+    stream.synchronize()
+    c0 = dg.dg_launch_count()
+    g1, g2 = [], []
+    for k in range(period):
+        a, b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(a, stream=stream):
+            k1(k)
+        with torch.cuda.graph(b, stream=stream):
+            k2(k)
+        g1.append(a)
+        g2.append(b)
+    launches_per_step = (dg.dg_launch_count() - c0) / period
+    assert dg.dg_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            g1[k % period].replay()
+            g2[k % period].replay()
+    stream.synchronize()
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for k in range(K):
+                j = (args.warmup + k) % period
+                g1[j].replay()
+                ev[2 * k + 1].record(stream)
+                g2[j].replay()
+                ev[2 * k + 2].record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier()
+    total_ms = ev[0].elapsed_time(ev[2 * K])
+    k1_us = [ev[2 * k].elapsed_time(ev[2 * k + 1]) * 1e3 for k in range(K)]
+    k2_us = [ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) * 1e3 for k in range(K)]
+    dev_err = dg.dg_device_error()
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    steps_per_s = world * K / (total_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (the contraction) and of the logits pass
+    k1_mean = statistics.mean(k1_us)
+    k2_mean = statistics.mean(k2_us)
+    flops_k2 = 2.0 * cfg.R * cfg.V * cfg.d
+    bytes_k2 = cfg.V * cfg.d * 2 + cfg.R * cfg.V * 2 + cfg.R * cfg.d * 2 + cfg.R * 4
+    bytes_k1 = cfg.R * cfg.V * 2 + cfg.R * 4 + cfg.R * 25
+    hbm = peaks["hbm_gbs"]
+    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_tensor_us = flops_k2 / (tc * 1e12) * 1e6
+    t_hbm_us = bytes_k2 / (hbm * 1e9) * 1e6
+    if t_tensor_us >= t_hbm_us:
+        achieved = flops_k2 / (k2_mean * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc, "unit": "TFLOP/s",
+                "frac": round(achieved / tc, 4)}
+    else:
+        achieved = bytes_k2 / (k2_mean * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4)}
+    roof["traffic"] = traffic_from_profiles("selfcond.cu", "selfcond_full_vocab.md")
+    roof["kernel"] = "selfcond (z = softmax(L) E, tcgen05)"
+    roof["peak_source"] = f"{peaks['source']} ({'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} bf16)"
+    roof["slower_bound_us"] = round(max(t_tensor_us, t_hbm_us), 1)
+    roof["frac_of_slower_bound"] = round(max(t_tensor_us, t_hbm_us) / k2_mean, 4)
+    k1_gbs = bytes_k1 / (k1_mean * 1e-6) / 1e9
+
+    # ---- training-side kernels on the training workload (forward noise + canvas CE)
+    train = bench_train(dg, W, dev, stream, hbm)
+
+    # ---- end to end through the public API with host buffers
+    e2e = bench_e2e(dg, W, cfg, dev, E, args, world, barrier)
+
+    line = {
+        "metric": METRIC,
+        "value": round(steps_per_s, 2),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; logits N(0,1.5) + Zipf(1.1) boost on 64 ids per row; E ~ N(0, 0.02))",
+        "config": {"workload": "full-vocab sampler step: 1 canvas, C=256, V=262144, d=2048, bf16, cosine, "
+                               "12 steps per block; step = logits pass + self-conditioning contraction",
+                   "B": cfg.B, "C": cfg.C, "V": cfg.V, "d": cfg.d, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {nbuf} rotating logits buffers of {lbytes / 1e6:.1f} MB "
+                         f"+ E {cfg.V * cfg.d * 2 / 1e9:.2f} GB"},
+        "canvas_tokens_per_s": round(steps_per_s * cfg.C, 1),
+        "roofline": roof,
+        "kernels": {
+            "logits_pass_us": round(k1_mean, 2), "logits_pass_GBps": round(k1_gbs, 1),
+            "logits_pass_frac_hbm": round(k1_gbs / hbm, 4),
+            "selfcond_us": round(k2_mean, 2),
+            "selfcond_TFLOPs": round(flops_k2 / (k2_mean * 1e-6) / 1e12, 1),
+            "selfcond_frac_tensor_sustained": round(flops_k2 / (k2_mean * 1e-6) / 1e12 / tc, 4),
+            "selfcond_frac_hbm": round(bytes_k2 / (k2_mean * 1e-6) / 1e9 / hbm, 4),
+            "train": train,
+        },
+        "e2e": e2e,
+        "gpu_launches": int(round(launches_per_step * K)),
+        "device_error": dev_err,
+        "clocks": clocks.summary(),
+    }
+    return line
+
+
+def bench_train(dg, W, dev, stream, hbm):
+    import torch
+    cfg = W.TRAIN
+    x0 = W.make_train_tokens(cfg, dev)
+    t = W.make_train_times(cfg)
+    logits = W.make_train_logits(cfg, dev)
+    xt = torch.empty_like(x0)
+    kidx = torch.empty(cfg.n_seq, dtype=torch.int32, device=dev)
+    loss = torch.empty(cfg.n_seq * cfg.C, dtype=torch.float32, device=dev)
+    seq = torch.empty(cfg.n_seq, dtype=torch.float32, device=dev)
+    lse = torch.empty_like(loss)
+    ws = torch.zeros(dg.dg_canvas_ce_workspace_size(cfg.n_seq, cfg.C, cfg.V), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        gn, gc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        dg.dg_forward_noise(x0, cfg.P, cfg.K, cfg.C, cfg.V, t, seed=1, x_t=xt, canvas_idx=kidx, stream=stream)
+        dg.dg_canvas_ce(logits, x0, kidx, cfg.P, cfg.K, cfg.C, loss_rows=loss, loss_seq=seq, lse_rows=lse, ws=ws,
+                        stream=stream)
+    stream.synchronize()
+    with torch.cuda.graph(gn, stream=stream):
+        dg.dg_forward_noise(x0, cfg.P, cfg.K, cfg.C, cfg.V, t, seed=1, x_t=xt, canvas_idx=kidx, stream=stream)
+    with torch.cuda.graph(gc, stream=stream):
+        dg.dg_canvas_ce(logits, x0, kidx, cfg.P, cfg.K, cfg.C, loss_rows=loss, loss_seq=seq, lse_rows=lse, ws=ws,
+                        stream=stream)
+    reps = 20
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gn.replay()
+            gc.replay()
+        e[0].record(stream)
+        for _ in range(reps):
+            gn.replay()
+        e[1].record(stream)
+        for _ in range(reps):
+            gc.replay()
+        e[2].record(stream)
+    stream.synchronize()
+    noise_us = e[0].elapsed_time(e[1]) * 1e3 / reps
+    ce_us = e[1].elapsed_time(e[2]) * 1e3 / reps
+    ce_bytes = cfg.n_seq * cfg.C * cfg.V * 2
+    return {"workload": "train: 8 seq x (P=512 + K=4 x C=256), V=262144, bf16 CE logits [2048, 262144]",
+            "forward_noise_us": round(noise_us, 2), "canvas_ce_us": round(ce_us, 2),
+            "canvas_ce_GBps": round(ce_bytes / (ce_us * 1e-6) / 1e9, 1),
+            "canvas_ce_frac_hbm": round(ce_bytes / (ce_us * 1e-6) / 1e9 / hbm, 4),
+            "note": "canvas CE logits (1.07 GB) exceed L2; repeated on one buffer"}
+
+
+def bench_e2e(dg, W, cfg, dev, E, args, world, barrier):
+    """Same metric through the public API with host buffers: every step copies its logits from
+    pinned host memory to the device and reads x_next and z back into pinned host memory."""
+    import torch
+    host_logits = W.make_logits(cfg, "cpu").pin_memory()
+    dev_logits = torch.empty_like(host_logits, device=dev)
+    x_t = W.make_canvas(cfg, dev)
+    host_x = torch.empty(cfg.R, dtype=torch.int32).pin_memory()
+    host_z = torch.empty((cfg.R, cfg.d), dtype=torch.bfloat16).pin_memory()
+    stream = torch.cuda.Stream(device=dev)
+    steps = max(3, min(args.steps, 24))
+
+    def one(k):
+        dev_logits.copy_(host_logits, non_blocking=True)
+        t, dt = cfg.times(k % cfg.steps)
+        out = dg.dg_sampler_step(dev_logits, x_t, cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=k, stream=stream)
+        z = dg.dg_selfcond(dev_logits, E, cfg.C, lse=out["lse"], stream=stream)
+        x_t.copy_(out["x_next"])
+        host_x.copy_(out["x_next"], non_blocking=True)
+        host_z.copy_(z, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for k in range(3):
+            one(k)
+    stream.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(steps):
+            one(k)
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * steps / (ms / 1e3), 2), "unit": "steps/s",
+            "h2d_bytes_per_step": host_logits.numel() * host_logits.element_size(),
+            "d2h_bytes_per_step": host_x.numel() * 4 + host_z.numel() * 2, "steps": steps}
+
+
+# ------------------------------------------------------------------------------ the oracle
+class OracleSample:
+    """The CPU oracle (plain single-threaded C, double precision, as it stands) on a bounded sample
+    of the full-vocab workload: the logits-pass work (statistics, argmax, two-level draw, Step)
+    on `rows1` rows and the contraction z = softmax(l) E on `rows2` rows over a fraction
+    `vfrac` of the vocabulary; the measured time is scaled to one step (256 rows, all of V)."""
+
+    def __init__(self, rows1: int, rows2: int, vfrac: int):
+        import numpy as np
+        from discrete_diffusion_lm_b200 import workloads as W
+        self.cfg = cfg = W.FULL
+        self.rows1, self.rows2, self.vfrac = rows1, rows2, vfrac
+        n = max(rows1, rows2)
+        self.L = W.make_logits(cfg, "cpu", rows=n).float().numpy()
+        self.Vs = cfg.V // vfrac
+        self.E = W.make_embedding(cfg, "cpu")[: self.Vs].float().numpy()
+        self.Ls = np.ascontiguousarray(self.L[:rows2, : self.Vs])
+        self.x_t = np.zeros(rows1, dtype=np.int32)
+
+    def run(self) -> dict:
+        from oracle import oracle as O
+        cfg = self.cfg
+        t, dt = cfg.times(0)
+        t0 = time.perf_counter()
+        O.sampler_step(self.L[: self.rows1], self.x_t, 1, self.rows1, cfg.V, cfg.schedule, t[:1], dt[:1], None, 0, 0,
+                       "sample")
+        t1 = time.perf_counter()
+        O.selfcond_rows(self.Ls, self.E, list(range(self.rows2)))
+        t2 = time.perf_counter()
+        step_s = cfg.R * ((t1 - t0) / self.rows1 + (t2 - t1) * self.vfrac / self.rows2)
+        return {"value": 1.0 / step_s, "unit": "steps/s", "cores": 1, "kind": "oracle", "cpu_seconds": t2 - t0,
+                "sample": f"full-vocab workload: logits pass on {self.rows1} rows of V=262144 + z on "
+                          f"{self.rows2} rows over 1/{self.vfrac} of V, scaled to 256 rows x full V per step"}
+
+
+def oracle_baseline() -> dict:
+    """About 10-20 s of single-threaded oracle work on rank 0."""
+    r = OracleSample(rows1=256, rows2=24, vfrac=1).run()
+    r["value"] = round(r["value"], 6)
+    r["cpu_seconds"] = round(r["cpu_seconds"], 1)
+    return r
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, one bounded sample per step."""
+    if rank != 0:
+        return None
+    samp = OracleSample(rows1=4, rows2=1, vfrac=8)
+    for _ in range(args.warmup):
+        samp.run()
+    res = [samp.run() for _ in range(args.steps)]
+    secs = sum(1.0 / r["value"] for r in res)  # extrapolated seconds for K full steps
+    v = args.steps / secs
+    cfg = samp.cfg
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / v, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": "full-vocab sampler step: 1 canvas, C=256, V=262144, d=2048, bf16, cosine, "
+                                   "12 steps per block; step = logits pass + self-conditioning contraction",
+                       "B": cfg.B, "C": cfg.C, "V": cfg.V, "d": cfg.d},
+            "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": 1, "kind": "oracle",
+                             "sample": res[0]["sample"]},
+            "e2e": {"value": round(v, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=120)
+    ap.add_argument("--warmup", type=int, default=12)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                             timeout=__import__("datetime").timedelta(seconds=120))
+    line = run_ours(args, rank, world, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline()
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
