@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.dg_sampler_step_workspace_size.restype = _sz
         L.dg_sampler_step.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32, _int,
                                       _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]
+        L.dg_sampler_step_noalloc.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32,
+                                              _int, _p, _p, _p, _p, _p, _p, _p, _p]
         L.dg_selfcond_workspace_size.argtypes = [_i32, _i32, _i32, _int, _int, _int]
         L.dg_selfcond_workspace_size.restype = _sz
         L.dg_selfcond.argtypes = [_p, _int, _i64, _i32, _i32, _i32, _p, _p, _p, _int, _i32, _p, _p, _sz, _p]
@@ -200,6 +202,40 @@ def dg_sampler_step(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V
         _ptr(out.get("lse")), _ptr(out.get("entropy")), _ptr(out.get("branch")),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("dg_sampler_step", rc)
+    return out
+
+
+DG_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
+
+
+def dg_sampler_step_noalloc(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V: Optional[int] = None,
+                            schedule: str = "cosine", inv_tau=None, seed: int = 0, step: int = 0,
+                            mode: str = "sample", out: Optional[dict] = None, stream=None) -> dict:
+    """The sampler step without a caller workspace: for callers that cannot allocate device
+    memory where they sample.  Scratch lives in the library's fixed device array (at most
+    DG_NOALLOC_SCRATCH_BYTES); calls share it, so overlapping calls race.  Output tensors are
+    the caller's (pass `out` to reuse buffers; otherwise they are created here, as for
+    dg_sampler_step)."""
+    ld = _row_major_2d(logits, "logits")
+    R = logits.shape[0]
+    V = logits.shape[1] if V is None else V
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = logits.device
+    if out is None:
+        out = {k: torch.empty(R, dtype=dt_, device=dev) for k, dt_ in
+               (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32),
+                ("max_prob", torch.float32), ("lse", torch.float32), ("entropy", torch.float32),
+                ("branch", torch.uint8))}
+    rc = lib().dg_sampler_step_noalloc(
+        _ptr(logits), _dtype_code(logits), ld, _ptr(x_t), B, C, V, DG_SCHED[schedule],
+        _host_doubles(_expand(t, B), B), _host_doubles(_expand(dt, B), B),
+        _host_floats(None if inv_tau is None else _expand(inv_tau, B), B),
+        ctypes.c_uint64(seed), ctypes.c_uint32(step), DG_X0[mode],
+        _ptr(out.get("x_next")), _ptr(out.get("x0_hat")), _ptr(out.get("argmax")), _ptr(out.get("max_prob")),
+        _ptr(out.get("lse")), _ptr(out.get("entropy")), _ptr(out.get("branch")), _stream(stream))
+    _check("dg_sampler_step_noalloc", rc)
     return out
 
 

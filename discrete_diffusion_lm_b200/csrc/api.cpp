@@ -160,6 +160,8 @@ int check_inv_tau(const float* inv_tau, int32_t B, float* out) {
 
 void note_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+void set_error_message(int /*code*/, const char* msg) { g_last_error = msg ? msg : ""; }
+
 }  // namespace dg
 
 using namespace dg;

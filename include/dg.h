@@ -174,6 +174,36 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
                  int32_t V, float* loss_rows, float* loss_seq, float* lse_rows, void* workspace,
                  size_t workspace_bytes, dg_stream_t stream);
 
+/* ------------------------------------------------------------------------ */
+/* Allocation-free sampler step.  The pages have no counterpart: this entry  */
+/* point exists for callers that cannot allocate device memory where they   */
+/* sample (a serving loop that must not call cudaMalloc, which can stall the */
+/* whole device; a runtime that owns all device memory and passes the       */
+/* library only input and output buffers).  It computes exactly what        */
+/* dg_sampler_step computes, with the same arguments except the workspace: */
+/* the scratch lives in a fixed device array of DG_NOALLOC_SCRATCH_BYTES     */
+/* that every GPU loading the library holds until the process exits.        */
+/*   - Limit: B*C rows of V ids must fit, i.e.                               */
+/*     dg_sampler_step_workspace_size(B*C, V) <= DG_NOALLOC_SCRATCH_BYTES     */
+/*     (256 rows of V = 262144 take about 2 MiB); larger requests return     */
+/*     DG_ERR_WORKSPACE before anything is enqueued.                         */
+/*   - The first call on a device looks up the array's device address       */
+/*     (cudaGetSymbolAddress) with that device current; make that first call */
+/*     before any stream capture on the device.                              */
+/*   - Each call clears the part of the array it uses (an async memset on    */
+/*     `stream`), so earlier contents never matter; all calls share the one  */
+/*     array, so calls that overlap on the GPU race: serialise them (one     */
+/*     stream, or events).  No call allocates or frees device memory.         */
+/* ------------------------------------------------------------------------ */
+#define DG_NOALLOC_SCRATCH_BYTES (4 * 1024 * 1024)
+
+int dg_sampler_step_noalloc(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t,
+                            int32_t B, int32_t C, int32_t V, int schedule, const double* t,
+                            const double* dt, const float* inv_tau, uint64_t seed, uint32_t step,
+                            int x0_mode, int32_t* x_next, int32_t* x0_hat, int32_t* argmax,
+                            float* max_prob, float* lse, float* entropy, uint8_t* branch,
+                            dg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
