@@ -36,7 +36,8 @@ namespace {
 
 constexpr int kKBlock = 32;  // vocabulary ids per pipeline stage
 constexpr int kTileM = 128;  // rows per CTA = TMEM lanes
-constexpr int kNumSoftmaxWarps = 4;
+constexpr int kNumSoftmaxWarps = 8;  // two groups of four; group g converts the stages i with i % 2 == g
+constexpr int kGroupThreads = 128;
 constexpr int kThreads = 64 + 32 * kNumSoftmaxWarps;  // producer warp, MMA warp, softmax warps
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at the boost clock
 
@@ -117,6 +118,21 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
             "r"(smem_u32(dst)),
         "l"(tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
+}
+// Barrier among the four warps of one softmax group (named barrier 1 + group, 128 threads) that
+// also ORs a flag over them, so that every thread of the group takes the same exit decision (a
+// partial arrival would hang).
+__device__ __forceinline__ bool softmax_group_sync_or(int group, bool flag) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(flag)), "r"(1 + group), "n"(kGroupThreads)
+        : "memory");
+    return r != 0;
 }
 __device__ __forceinline__ void tcgen05_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tcgen05_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -211,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&efull[s], 1);
             mbar_init(&lfull[s], 1);
-            mbar_init(&pready[s], 32 * kNumSoftmaxWarps);
+            mbar_init(&pready[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
@@ -293,18 +309,20 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ..
+        const int group = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const int32_t r = mt * kTileM + row;
         const bool valid = r < p.R;
         const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
         const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
-        for (int i = 0; i < nkb; ++i) {
+        for (int i = group; i < nkb; i += 2) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
-            if (!mbar_wait(&lfull[s], ph, abort_flag)) break;
+            const bool ok = mbar_wait(&lfull[s], ph, abort_flag);
             uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
-            if (kBf16) {
+            if (!ok) {
+            } else if (kBf16) {
                 // row of 32 bf16 = 64 bytes; 16-byte chunk j stored at j ^ ((row >> 1) & 3)
                 uint8_t* rb = lt + row * 64;
                 const int sw = (row >> 1) & 3;
@@ -330,13 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                     *reinterpret_cast<uint4*>(pb + ((q ^ sw4) << 4)) = o;
                 }
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&pready[s]);
+            fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
+            if (softmax_group_sync_or(group, !ok)) break;
+            if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);
         }
-        if (mbar_wait(accum, 0, abort_flag)) {
+        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, abort_flag))) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            for (int c = 0; c < kNT; c += 32) {
+            for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(lane_base + c, v);
                 if (valid) {
@@ -370,6 +389,316 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
     tcgen05_after_sync();
     if (warp == 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(static_cast<uint32_t>(kNT))
+                     : "memory");
+}
+
+// ------------------------------------------------------------------------------------ CTA-pair form
+// For 129 rows or more, a cluster of two CTAs shares each tile: tcgen05.mma.cta_group::2 with
+// M = 256 reads A (p) from both CTAs -- 128 rows each, from their own shared memory -- and B (E)
+// split by columns: each CTA stages only the half of every 256-column block that belongs to it,
+// so per 32-id stage a CTA loads 16 KB of E instead of 32 KB and the pipeline gets 8 stages.
+// The pair's accumulator is 128 TMEM lanes x kNT columns in each CTA (its own rows).
+// Signalling: both CTAs' E copies complete on the leader CTA's barrier (cta_group::2 TMA, no
+// multicast); the peer's softmax warps arrive remotely on the leader's p-ready barrier; the
+// leader's MMA thread commits each stage to its own and to its peer's empty barrier.
+
+template <bool kBf16, int kNT>
+struct PairCfg {
+    static constexpr int kMmaN = kNT > 256 ? 256 : kNT;
+    static constexpr int kBoxesPerHalf = kMmaN / 128;  // 64-column boxes per CTA per MMA block
+    static constexpr uint32_t kEBytes = (kNT / 2) * kKBlock * 2;
+    static constexpr uint32_t kLBytes = kTileM * kKBlock * (kBf16 ? 2 : 4);
+    static constexpr uint32_t kPBytes = kBf16 ? 0 : kTileM * kKBlock * 2;
+    static constexpr uint32_t kStageBytes = kEBytes + kLBytes + kPBytes;
+    static constexpr int kStagesFit = static_cast<int>((200u * 1024u) / kStageBytes);
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr uint32_t kBarrierBytes = 512;
+    static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+    static_assert(kNT >= 128 && kNT % 128 == 0, "pair tiles hold whole 64-column boxes per CTA");
+    static_assert(kStages >= 3, "pipeline needs three stages");
+    static_assert(kEBytes % 1024 == 0 && kLBytes % 1024 == 0 && kPBytes % 1024 == 0, "1 KB-aligned stage parts");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrival on a barrier of another CTA of the cluster (default release semantics).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (arrivals may come from the other CTA of the pair).
+__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_device_error, 1);
+            return false;
+        }
+    }
+}
+// E box copy whose completion is counted on the pair leader's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* tm, int32_t c0, int32_t c1,
+                                                 uint32_t leader_bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(tm), "r"(c0), "r"(c1), "r"(leader_bar)
+        : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
+template <bool kBf16, int kNT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    selfcond_pair_kernel(const __grid_constant__ KernelParams p) {
+    using G = PairCfg<kBf16, kNT>;
+    constexpr int kStages = G::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* efull = reinterpret_cast<uint64_t*>(smem + kStages * G::kStageBytes);  // leader's: both E halves
+    uint64_t* lfull = efull + kStages;   // own logits landed
+    uint64_t* pready = lfull + kStages;  // leader's: p written by both CTAs (one arrival per warp)
+    uint64_t* empty = pready + kStages;  // own stage free again (leader's commit)
+    uint64_t* accum = empty + kStages;   // own accumulator final (leader's commit)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const uint32_t rank = cluster_rank();
+    int bid = blockIdx.x >> 1;  // pair index
+    const int split = bid % p.splits;
+    bid /= p.splits;
+    const int nt = bid % p.n_tiles;
+    const int mp = bid / p.n_tiles;  // pair of 128-row tiles: rows 256 mp .. 256 mp + 255
+    const int kb0 = static_cast<int>(static_cast<long long>(split) * p.total_kb / p.splits);
+    const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.total_kb / p.splits);
+    const int nkb = kb1 - kb0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&efull[s], 1);
+            mbar_init(&lfull[s], 1);
+            // leader: one arrival from each CTA of the pair; peer: its own softmax warps (forwarded)
+            mbar_init(&pready[s], rank == 0 ? 2 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accum, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(static_cast<uint32_t>(kNT))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tcgen05_before_sync();
+    cluster_sync();  // barriers of both CTAs initialised before any remote arrival
+    tcgen05_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer (both CTAs)
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
+                uint8_t* st = smem + s * G::kStageBytes;
+                const int32_t k0 = (kb0 + i) * kKBlock;
+                mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
+                tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mp * 2 * kTileM + static_cast<int>(rank) * kTileM,
+                            &lfull[s]);
+                if (rank == 0) mbar_arrive_expect_tx(&efull[s], 2 * G::kEBytes);
+                const uint32_t leader_bar = map_to_rank(smem_u32(&efull[s]), 0);
+#pragma unroll
+                for (int nh = 0; nh < kNT / G::kMmaN; ++nh)
+#pragma unroll
+                    for (int j = 0; j < G::kBoxesPerHalf; ++j) {
+                        const int col = nt * kNT + nh * G::kMmaN + static_cast<int>(rank) * (G::kMmaN / 2) + 64 * j;
+                        tma_load_2d_pair(st + (nh * G::kBoxesPerHalf + j) * (64 * kKBlock * 2), &p.tm_E, col, k0,
+                                         leader_bar);
+                    }
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i) {
+                    const int s = i % kStages;
+                    const uint32_t ph = (i / kStages) & 1;
+                    const long long t0 = clock64();
+                    while (!(mbar_try_wait(&lfull[s], ph) && (rank != 0 || mbar_try_wait(&efull[s], ph))) &&
+                           clock64() - t0 < kWaitLimitCycles) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1 && rank == 1) {
+        // ---------------------------------------------------------------- p-ready forwarder (peer)
+        // Passes "p of stage s is written" on to the leader with a cluster-scope release, off the
+        // softmax warps' critical path.
+        if (lane == 0) {
+            const uint32_t leader_pready0 = map_to_rank(smem_u32(&pready[0]), 0);
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                mbar_arrive_remote(leader_pready0 + s * 8);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (leader)
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(2 * kTileM, G::kMmaN);
+            const uint32_t peer_empty0 = map_to_rank(smem_u32(&empty[0]), 1);
+            const uint32_t own_empty0 = map_to_rank(smem_u32(&empty[0]), 0);
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&efull[s], ph, abort_flag)) break;
+                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                tcgen05_after_sync();
+                uint8_t* st = smem + s * G::kStageBytes;
+                const uint32_t a_base = smem_u32(st + G::kEBytes + (kBf16 ? 0 : G::kLBytes));
+                const uint32_t b_base = smem_u32(st);
+#pragma unroll
+                for (int ks = 0; ks < kKBlock / 16; ++ks) {
+                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 512, kLayoutSw64);
+#pragma unroll
+                    for (int nh = 0; nh < kNT / G::kMmaN; ++nh) {
+                        const uint64_t bdesc = smem_desc(
+                            b_base + nh * G::kBoxesPerHalf * (64 * kKBlock * 2) + ks * 2048, 64 * kKBlock * 2, 1024,
+                            kLayoutSw128);
+                        umma_bf16_pair(tmem + nh * G::kMmaN, adesc, bdesc, idesc, (i > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit_pair(own_empty0 + s * 8);
+                umma_commit_pair(peer_empty0 + s * 8);
+            }
+            umma_commit_pair(map_to_rank(smem_u32(accum), 0));
+            umma_commit_pair(map_to_rank(smem_u32(accum), 1));
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax + epilogue (both CTAs)
+        const int quarter = warp & 3;
+        const int group = (warp - 2) >> 2;
+        const int row = quarter * 32 + lane;
+        const int32_t r = mp * 2 * kTileM + static_cast<int>(rank) * kTileM + row;
+        const bool valid = r < p.R;
+        const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
+        const float a = it * kLog2e;
+        const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
+        for (int i = group; i < nkb; i += 2) {
+            const int s = i % kStages;
+            const uint32_t ph = (i / kStages) & 1;
+            const bool ok = mbar_wait(&lfull[s], ph, abort_flag);
+            uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
+            if (!ok) {
+            } else if (kBf16) {
+                uint8_t* rb = lt + row * 64;
+                const int sw = (row >> 1) & 3;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4* q = reinterpret_cast<uint4*>(rb + ((j ^ sw) << 4));
+                    *q = softmax_chunk_bf16(*q, a, nb);
+                }
+            } else {
+                const uint8_t* rb = lt + row * 128;
+                uint8_t* pb = lt + G::kLBytes + row * 64;
+                const int sw8 = row & 7, sw4 = (row >> 1) & 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 c0 = *reinterpret_cast<const uint4*>(rb + (((2 * q) ^ sw8) << 4));
+                    const uint4 c1 = *reinterpret_cast<const uint4*>(rb + (((2 * q + 1) ^ sw8) << 4));
+                    uint4 o;
+                    o.x = softmax_pair_f32(c0.x, c0.y, a, nb);
+                    o.y = softmax_pair_f32(c0.z, c0.w, a, nb);
+                    o.z = softmax_pair_f32(c1.x, c1.y, a, nb);
+                    o.w = softmax_pair_f32(c1.z, c1.w, a, nb);
+                    *reinterpret_cast<uint4*>(pb + ((q ^ sw4) << 4)) = o;
+                }
+            }
+            fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
+            if (softmax_group_sync_or(group, !ok)) break;
+            if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);  // local; the peer's is forwarded by warp 1
+        }
+        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, abort_flag))) {
+            tcgen05_after_sync();
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(lane_base + c, v);
+                if (valid) {
+                    const int32_t col = nt * kNT + c;
+                    if (p.splits == 1) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.z + static_cast<size_t>(r) * p.d + col);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                            dst[q] = o;
+                        }
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.partial + (static_cast<size_t>(split) * p.R + r) * p.d + col);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    // Neither CTA leaves (or frees TMEM) while its peer may still touch its shared memory or the
+    // pair's accumulator.
+    tcgen05_before_sync();
+    __syncthreads();
+    cluster_sync();
+    tcgen05_after_sync();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(static_cast<uint32_t>(kNT))
                      : "memory");
 }
 
@@ -443,16 +772,33 @@ int num_sms() {
     return v;
 }
 
-// Split the vocabulary so that the grid is about one wave of CTAs (one CTA per SM).
-void plan(int R, int V, int d, int* m_tiles, int* n_tiles, int* splits, int* total_kb) {
-    *m_tiles = (R + kTileM - 1) / kTileM;
-    *n_tiles = d / pick_ntile(d);
-    *total_kb = (V + kKBlock - 1) / kKBlock;
-    const int tiles = *m_tiles * *n_tiles;
-    int s = num_sms() / tiles;
+// Work plan: CTA pairs (M = 256 per pair) when there are more than 128 rows and the column tile
+// is at least 128 wide, single CTAs otherwise; the vocabulary is split so that the grid is about
+// one wave (one CTA per SM).
+struct Plan {
+    bool pair;
+    int m_tiles;   // 128-row tiles (single) or 256-row pair tiles
+    int n_tiles;
+    int splits;
+    int total_kb;
+    int ctas;
+};
+
+Plan plan(int R, int V, int d) {
+    Plan pl;
+    const int nt = pick_ntile(d);
+    pl.pair = R > kTileM && nt >= 128;
+    pl.m_tiles = pl.pair ? (R + 2 * kTileM - 1) / (2 * kTileM) : (R + kTileM - 1) / kTileM;
+    pl.n_tiles = d / nt;
+    pl.total_kb = (V + kKBlock - 1) / kKBlock;
+    const int units = pl.m_tiles * pl.n_tiles;
+    const int per_unit = pl.pair ? 2 : 1;
+    int s = num_sms() / (per_unit * units);
     if (s < 1) s = 1;
-    if (s > *total_kb) s = *total_kb;
-    *splits = s;
+    if (s > pl.total_kb) s = pl.total_kb;
+    pl.splits = s;
+    pl.ctas = per_unit * units * s;
+    return pl;
 }
 
 template <bool kBf16, int kNT>
@@ -469,20 +815,33 @@ cudaError_t launch_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <bool kBf16, int kNT>
+cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
+    using G = PairCfg<kBf16, kNT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(selfcond_pair_kernel<kBf16, kNT>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::kSmemBytes));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    selfcond_pair_kernel<kBf16, kNT><<<grid, kThreads, G::kSmemBytes, st>>>(kp);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d) {
-    int mt, ntl, s, tkb;
     if (R < 1 || V < 1 || d < 64) return 0;
-    plan(R, V, d, &mt, &ntl, &s, &tkb);
-    return s > 1 ? static_cast<size_t>(s) * R * d * sizeof(float) : 0;
+    const Plan pl = plan(R, V, d);
+    return pl.splits > 1 ? static_cast<size_t>(pl.splits) * R * d * sizeof(float) : 0;
 }
 
 cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     static thread_local KernelParams kp;
     std::memset(&kp, 0, sizeof(kp));
-    int m_tiles, n_tiles, splits, total_kb;
-    plan(sp.R, sp.V, sp.d, &m_tiles, &n_tiles, &splits, &total_kb);
+    const Plan pl = plan(sp.R, sp.V, sp.d);
+    const int splits = pl.splits;
     const int nt = pick_ntile(sp.d);
     cudaError_t e;
     if (sp.logits_bf16)
@@ -502,13 +861,24 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     kp.C = sp.C;
     kp.V = sp.V;
     kp.d = sp.d;
-    kp.n_tiles = n_tiles;
+    kp.n_tiles = pl.n_tiles;
     kp.splits = splits;
-    kp.total_kb = total_kb;
+    kp.total_kb = pl.total_kb;
     std::memcpy(kp.inv_tau, sp.inv_tau, sizeof(kp.inv_tau));
-    const int grid = m_tiles * n_tiles * splits;
+    const int grid = pl.ctas;
 #define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st)
-    if (sp.logits_bf16) {
+#define DG_PC(BF, NT) e = launch_pair_kernel<BF, NT>(kp, grid, st)
+    if (pl.pair) {
+        if (sp.logits_bf16) {
+            if (nt == 512) DG_PC(true, 512);
+            else if (nt == 256) DG_PC(true, 256);
+            else DG_PC(true, 128);
+        } else {
+            if (nt == 512) DG_PC(false, 512);
+            else if (nt == 256) DG_PC(false, 256);
+            else DG_PC(false, 128);
+        }
+    } else if (sp.logits_bf16) {
         if (nt == 512) DG_SC(true, 512);
         else if (nt == 256) DG_SC(true, 256);
         else if (nt == 128) DG_SC(true, 128);
@@ -520,6 +890,7 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
         else DG_SC(false, 64);
     }
 #undef DG_SC
+#undef DG_PC
     note_launches(1);
     if (e != cudaSuccess || splits == 1) return e;
     const int64_t n4 = static_cast<int64_t>(sp.R) * sp.d / 4;
