@@ -218,9 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
     bid /= p.splits;
     const int nt = bid % p.n_tiles;
     const int mt = bid / p.n_tiles;
-    const int kb0 = static_cast<int>(static_cast<long long>(split) * p.total_kb / p.splits);
-    const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.total_kb / p.splits);
-    const int nkb = kb1 - kb0;
+    // Split s takes the 32-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
+    // few rows of E, so every E row is fetched by all its readers within a short window.
+    const int kb0 = split;
+    const int kstride = p.splits;
+    const int nkb = (p.total_kb - split + p.splits - 1) / p.splits;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -254,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                 const uint32_t ph = (i / kStages) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
                 uint8_t* st = smem + s * G::kStageBytes;
-                const int32_t k0 = (kb0 + i) * kKBlock;
+                const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
                 tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mt * kTileM, &lfull[s]);
                 mbar_arrive_expect_tx(&efull[s], G::kEBytes);
@@ -409,15 +411,22 @@ struct PairCfg {
     static constexpr uint32_t kEBytes = (kNT / 2) * kKBlock * 2;
     static constexpr uint32_t kLBytes = kTileM * kKBlock * (kBf16 ? 2 : 4);
     static constexpr uint32_t kPBytes = kBf16 ? 0 : kTileM * kKBlock * 2;
-    static constexpr uint32_t kStageBytes = kEBytes + kLBytes + kPBytes;
-    static constexpr int kStagesFit = static_cast<int>((200u * 1024u) / kStageBytes);
-    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-    static constexpr uint32_t kBarrierBytes = 512;
-    static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+    static constexpr uint32_t kLStageBytes = kLBytes + kPBytes;
+    // A logits stage makes a long round trip (land, softmax, forward to the leader, MMA, release),
+    // so the logits ring needs about as much depth as the E ring even though its copies are fast.
+    static constexpr uint32_t kBudget = 212u * 1024u;
+    static constexpr int kLStagesFit = static_cast<int>((kBudget - 4 * kEBytes) / kLStageBytes);
+    static constexpr int kLStages = kLStagesFit > 8 ? 8 : kLStagesFit;
+    static constexpr int kEStagesFit = static_cast<int>((kBudget - kLStages * kLStageBytes) / kEBytes);
+    static constexpr int kEStages = kEStagesFit > 16 ? 16 : kEStagesFit;
+    static constexpr uint32_t kBarrierBytes = 1024;
+    static constexpr uint32_t kSmemBytes = kEStages * kEBytes + kLStages * kLStageBytes + kBarrierBytes + 1024;
     static_assert(kNT >= 128 && kNT % 128 == 0, "pair tiles hold whole 64-column boxes per CTA");
-    static_assert(kStages >= 3, "pipeline needs three stages");
+    static_assert(kEStages >= 4 && kLStages >= 2, "pipelines need depth");
     static_assert(kEBytes % 1024 == 0 && kLBytes % 1024 == 0 && kPBytes % 1024 == 0, "1 KB-aligned stage parts");
 };
+
+constexpr int kPairThreads = 96 + 32 * kNumSoftmaxWarps;  // E producer, MMA/forwarder, logits producer
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -486,17 +495,20 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
 }
 
 template <bool kBf16, int kNT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     selfcond_pair_kernel(const __grid_constant__ KernelParams p) {
     using G = PairCfg<kBf16, kNT>;
-    constexpr int kStages = G::kStages;
+    constexpr int kES = G::kEStages, kLS = G::kLStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* efull = reinterpret_cast<uint64_t*>(smem + kStages * G::kStageBytes);  // leader's: both E halves
-    uint64_t* lfull = efull + kStages;   // own logits landed
-    uint64_t* pready = lfull + kStages;  // leader's: p written by both CTAs (one arrival per warp)
-    uint64_t* empty = pready + kStages;  // own stage free again (leader's commit)
-    uint64_t* accum = empty + kStages;   // own accumulator final (leader's commit)
+    uint8_t* ering = smem;                             // kES x E half-tiles
+    uint8_t* lring = smem + kES * G::kEBytes;          // kLS x (logits tile [+ p tile])
+    uint64_t* efull = reinterpret_cast<uint64_t*>(lring + kLS * G::kLStageBytes);  // leader's: both halves
+    uint64_t* eempty = efull + kES;                    // own E stage free (leader's commit)
+    uint64_t* lfull = eempty + kES;                    // own logits landed
+    uint64_t* lempty = lfull + kLS;                    // own logits/p stage free (leader's commit)
+    uint64_t* pready = lempty + kLS;                   // leader: both CTAs' p; peer: own p (forwarded)
+    uint64_t* accum = pready + kLS;                    // own accumulator final
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -505,19 +517,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int split = bid % p.splits;
     bid /= p.splits;
     const int nt = bid % p.n_tiles;
-    const int mp = bid / p.n_tiles;  // pair of 128-row tiles: rows 256 mp .. 256 mp + 255
-    const int kb0 = static_cast<int>(static_cast<long long>(split) * p.total_kb / p.splits);
-    const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.total_kb / p.splits);
-    const int nkb = kb1 - kb0;
+    const int mp = bid / p.n_tiles;  // rows 256 mp .. 256 mp + 255; this CTA: 128 of them
+    // Split s takes the 32-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
+    // few rows of E, so every E row is fetched by all its readers within a short window.
+    const int kb0 = split;
+    const int kstride = p.splits;
+    const int nkb = (p.total_kb - split + p.splits - 1) / p.splits;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kFirstSoftmaxWarp = 3;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kES; ++s) {
             mbar_init(&efull[s], 1);
+            mbar_init(&eempty[s], 1);
+        }
+        for (int s = 0; s < kLS; ++s) {
             mbar_init(&lfull[s], 1);
-            // leader: one arrival from each CTA of the pair; peer: its own softmax warps (forwarded)
+            mbar_init(&lempty[s], 1);
             mbar_init(&pready[s], rank == 0 ? 2 : 1);
-            mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
         *abort_flag = 0;
@@ -535,51 +552,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer (both CTAs)
+        // ---------------------------------------------------------------- E producer (both CTAs)
         if (lane == 0) {
+            const uint32_t leader_efull0 = map_to_rank(smem_u32(&efull[0]), 0);
             int issued = 0;
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
-                uint8_t* st = smem + s * G::kStageBytes;
-                const int32_t k0 = (kb0 + i) * kKBlock;
-                mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
-                tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mp * 2 * kTileM + static_cast<int>(rank) * kTileM,
-                            &lfull[s]);
+                const int s = i % kES;
+                const uint32_t ph = (i / kES) & 1;
+                if (!mbar_wait(&eempty[s], ph ^ 1, abort_flag)) break;
+                const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 if (rank == 0) mbar_arrive_expect_tx(&efull[s], 2 * G::kEBytes);
-                const uint32_t leader_bar = map_to_rank(smem_u32(&efull[s]), 0);
+                uint8_t* dst = ering + s * G::kEBytes;
 #pragma unroll
                 for (int nh = 0; nh < kNT / G::kMmaN; ++nh)
 #pragma unroll
                     for (int j = 0; j < G::kBoxesPerHalf; ++j) {
                         const int col = nt * kNT + nh * G::kMmaN + static_cast<int>(rank) * (G::kMmaN / 2) + 64 * j;
-                        tma_load_2d_pair(st + (nh * G::kBoxesPerHalf + j) * (64 * kKBlock * 2), &p.tm_E, col, k0,
-                                         leader_bar);
+                        tma_load_2d_pair(dst + (nh * G::kBoxesPerHalf + j) * (64 * kKBlock * 2), &p.tm_E, col, k0,
+                                         leader_efull0 + s * 8);
                     }
                 issued = i + 1;
             }
-            if (*abort_flag) {
-                for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i) {
-                    const int s = i % kStages;
-                    const uint32_t ph = (i / kStages) & 1;
+            if (*abort_flag && rank == 0) {
+                // both halves of the last stages land on the leader's barriers: wait for them (bounded)
+                for (int i = issued - kES > 0 ? issued - kES : 0; i < issued; ++i) {
                     const long long t0 = clock64();
-                    while (!(mbar_try_wait(&lfull[s], ph) && (rank != 0 || mbar_try_wait(&efull[s], ph))) &&
-                           clock64() - t0 < kWaitLimitCycles) {
+                    while (!mbar_try_wait(&efull[i % kES], (i / kES) & 1) && clock64() - t0 < kWaitLimitCycles) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------------- logits producer (both CTAs)
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kLS;
+                const uint32_t ph = (i / kLS) & 1;
+                if (!mbar_wait(&lempty[s], ph ^ 1, abort_flag)) break;
+                const int32_t k0 = (kb0 + i * kstride) * kKBlock;
+                mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
+                tma_load_2d(lring + s * G::kLStageBytes, &p.tm_logits, k0,
+                            mp * 2 * kTileM + static_cast<int>(rank) * kTileM, &lfull[s]);
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                for (int i = issued - kLS > 0 ? issued - kLS : 0; i < issued; ++i) {
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(&lfull[i % kLS], (i / kLS) & 1) && clock64() - t0 < kWaitLimitCycles) {
                     }
                 }
             }
         }
     } else if (warp == 1 && rank == 1) {
         // ---------------------------------------------------------------- p-ready forwarder (peer)
-        // Passes "p of stage s is written" on to the leader with a cluster-scope release, off the
-        // softmax warps' critical path.
+        // Passes "p of stage s is written" on to the leader, off the softmax warps' critical path.
         if (lane == 0) {
             const uint32_t leader_pready0 = map_to_rank(smem_u32(&pready[0]), 0);
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                const int s = i % kLS;
+                if (!mbar_wait(&pready[s], (i / kLS) & 1, abort_flag)) break;
                 mbar_arrive_remote(leader_pready0 + s * 8);
             }
         }
@@ -587,17 +619,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- MMA issuer (leader)
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(2 * kTileM, G::kMmaN);
-            const uint32_t peer_empty0 = map_to_rank(smem_u32(&empty[0]), 1);
-            const uint32_t own_empty0 = map_to_rank(smem_u32(&empty[0]), 0);
+            const uint32_t eempty_own = map_to_rank(smem_u32(&eempty[0]), 0);
+            const uint32_t eempty_peer = map_to_rank(smem_u32(&eempty[0]), 1);
+            const uint32_t lempty_own = map_to_rank(smem_u32(&lempty[0]), 0);
+            const uint32_t lempty_peer = map_to_rank(smem_u32(&lempty[0]), 1);
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_wait(&efull[s], ph, abort_flag)) break;
-                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                const int es = i % kES, ls = i % kLS;
+                if (!mbar_wait(&efull[es], (i / kES) & 1, abort_flag)) break;
+                if (!mbar_wait(&pready[ls], (i / kLS) & 1, abort_flag)) break;
                 tcgen05_after_sync();
-                uint8_t* st = smem + s * G::kStageBytes;
-                const uint32_t a_base = smem_u32(st + G::kEBytes + (kBf16 ? 0 : G::kLBytes));
-                const uint32_t b_base = smem_u32(st);
+                const uint32_t a_base = smem_u32(lring + ls * G::kLStageBytes + (kBf16 ? 0 : G::kLBytes));
+                const uint32_t b_base = smem_u32(ering + es * G::kEBytes);
 #pragma unroll
                 for (int ks = 0; ks < kKBlock / 16; ++ks) {
                     const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 512, kLayoutSw64);
@@ -609,27 +641,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         umma_bf16_pair(tmem + nh * G::kMmaN, adesc, bdesc, idesc, (i > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit_pair(own_empty0 + s * 8);
-                umma_commit_pair(peer_empty0 + s * 8);
+                umma_commit_pair(eempty_own + es * 8);
+                umma_commit_pair(eempty_peer + es * 8);
+                umma_commit_pair(lempty_own + ls * 8);
+                umma_commit_pair(lempty_peer + ls * 8);
             }
             umma_commit_pair(map_to_rank(smem_u32(accum), 0));
             umma_commit_pair(map_to_rank(smem_u32(accum), 1));
         }
     } else {
         // ---------------------------------------------------------------- softmax + epilogue (both CTAs)
-        const int quarter = warp & 3;
-        const int group = (warp - 2) >> 2;
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int group = (warp - kFirstSoftmaxWarp) >> 2;
         const int row = quarter * 32 + lane;
         const int32_t r = mp * 2 * kTileM + static_cast<int>(rank) * kTileM + row;
         const bool valid = r < p.R;
         const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
         const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
+        const int leader_thread = (kFirstSoftmaxWarp + 4 * group) * 32;
         for (int i = group; i < nkb; i += 2) {
-            const int s = i % kStages;
-            const uint32_t ph = (i / kStages) & 1;
-            const bool ok = mbar_wait(&lfull[s], ph, abort_flag);
-            uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
+            const int s = i % kLS;
+            const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, abort_flag);
+            uint8_t* lt = lring + s * G::kLStageBytes;
             if (!ok) {
             } else if (kBf16) {
                 uint8_t* rb = lt + row * 64;
@@ -657,7 +691,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
             if (softmax_group_sync_or(group, !ok)) break;
-            if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);  // local; the peer's is forwarded by warp 1
+            if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
         }
         if (__all_sync(0xffffffffu, mbar_wait(accum, 0, abort_flag))) {
             tcgen05_after_sync();
@@ -825,7 +859,7 @@ cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::kSmemBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    selfcond_pair_kernel<kBf16, kNT><<<grid, kThreads, G::kSmemBytes, st>>>(kp);
+    selfcond_pair_kernel<kBf16, kNT><<<grid, kPairThreads, G::kSmemBytes, st>>>(kp);
     return cudaGetLastError();
 }
 
