@@ -52,7 +52,7 @@ struct PassParams {
     unsigned long long thr_stay_same[DG_MAX_CANVASES];  // x0_hat == x_t: stay if w0 < this
 };
 
-constexpr int kPassThreads = 256;
+constexpr int kPassThreads = 128;
 constexpr int kPassWarps = kPassThreads / 32;
 
 cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s);

@@ -168,6 +168,13 @@ struct MergeShared {
     int flag;
 };
 
+// Per-row merge, run by the last CTA of the row.  Global memory is visited in two round trips:
+// the chunk records (thread t holds the four consecutive chunks 4t .. 4t+3 in registers, so one
+// Philox call serves its four chunk Gumbel variates), then the two chunks that must be re-read
+// (the one holding the argmax and the level-1 winner), fetched together.  Rows of more than
+// 4 * kPassThreads chunks re-read their further records from L2 in each pass.
+static_assert(kChunk == 4 * kPassThreads, "one chunk is re-read as four ids per thread");
+
 template <bool kBf16, int kKind>
 __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t canvas, float inv_tau,
                                        const void* rowp, MergeShared& sh) {
@@ -176,18 +183,65 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const float4* rec = p.rec + static_cast<size_t>(row) * nch;
     const float nbig = neg_big(kBf16);
 
-    // Row statistics from the chunk records (log-sum-exp merge).
-    float mr = -INFINITY;
-    for (int32_t j = tid; j < nch; j += kPassThreads) mr = fmaxf(mr, ld_cg_f4(rec + j).x);
+    // Cross-entropy: the target logit is fetched alongside the records.
+    float target_logit = 0.f;
+    bool target_ok = false;
+    int32_t b_seq = 0, i_seq = 0;
+    if (kKind == kPassCE && tid == 0) {
+        b_seq = row / p.C;
+        i_seq = row - b_seq * p.C;
+        const int32_t k = p.canvas_idx[b_seq];
+        if (k >= 0 && k < p.K) {
+            const int32_t target =
+                p.x0[static_cast<int64_t>(b_seq) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i_seq];
+            if (target >= 0 && target < p.V) {
+                target_logit = load_logit(rowp, target, kBf16);
+                target_ok = true;
+            }
+        }
+    }
+
+    float4 r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int32_t j = 4 * tid + k;
+        r[k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    }
+    // Records beyond the first 4 * kPassThreads (rows longer than 262144 ids with 128 threads).
+    auto far_quad = [&](int32_t q, float4 (&f)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int32_t j = 4 * q + k;
+            f[k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        }
+    };
+
+    // Row maximum of the raw chunk maxima.
+    float mr = fmaxf(fmaxf(r[0].x, r[1].x), fmaxf(r[2].x, r[3].x));
+    for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
+        float4 f[4];
+        far_quad(q, f);
+        mr = fmaxf(mr, fmaxf(fmaxf(f[0].x, f[1].x), fmaxf(f[2].x, f[3].x)));
+    }
     const float m_raw = block_max<kPassWarps>(mr, sh.f);
     const float m_row = m_raw * inv_tau;
+
+    // Log-sum-exp merge of (S, T) relative to the row maximum.
     float s = 0.f, t = 0.f;
-    for (int32_t j = tid; j < nch; j += kPassThreads) {
-        const float4 r = ld_cg_f4(rec + j);
-        const float dm = r.x * inv_tau - m_row;
+    auto acc_st = [&](const float4& c) {
+        if (c.x == -INFINITY) return;  // missing chunk
+        const float dm = c.x * inv_tau - m_row;
         const float f = expf(dm);
-        s = fmaf(r.y, f, s);
-        t = fmaf(f, fmaf(r.y, dm, r.z), t);
+        s = fmaf(c.y, f, s);
+        t = fmaf(f, fmaf(c.y, dm, c.z), t);
+    };
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc_st(r[k]);
+    for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
+        float4 f[4];
+        far_quad(q, f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc_st(f[k]);
     }
     const float S = block_sum<kPassWarps>(s, sh.f);
     const float T = block_sum<kPassWarps>(t, sh.f);
@@ -203,29 +257,22 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     }
 
     if (kKind == kPassCE) {
-        const int32_t b = row / p.C;
-        const int32_t i = row - b * p.C;
         if (tid == 0) {
-            const int32_t k = p.canvas_idx[b];
-            float loss = __int_as_float(0x7fc00000);  // NaN for an out-of-range canvas or target
-            if (k >= 0 && k < p.K) {
-                const int32_t target =
-                    p.x0[static_cast<int64_t>(b) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i];
-                if (target >= 0 && target < p.V) loss = lse - load_logit(rowp, target, kBf16);
-            }
+            const float loss = target_ok ? lse - target_logit : __int_as_float(0x7fc00000);  // NaN: bad target
             p.loss_rows[row] = loss;
             if (p.lse) p.lse[row] = lse;
             p.row_ticket[row] = 0u;
             __threadfence();
-            const unsigned prev = atomicAdd(&p.seq_ticket[b], 1u);
+            const unsigned prev = atomicAdd(&p.seq_ticket[b_seq], 1u);
             sh.flag = prev == static_cast<unsigned>(p.C - 1);
+            sh.i[0] = b_seq;
         }
         __syncthreads();
         if (!sh.flag) return;
+        const int32_t b = sh.i[0];
         __threadfence();
         float acc = 0.f;
-        for (int32_t q = tid; q < p.C; q += kPassThreads)
-            acc += ld_cg_f(p.loss_rows + static_cast<int64_t>(b) * p.C + q);
+        for (int32_t q = tid; q < p.C; q += kPassThreads) acc += ld_cg_f(p.loss_rows + static_cast<int64_t>(b) * p.C + q);
         const float total = block_sum<kPassWarps>(acc, sh.f);
         if (tid == 0) {
             if (p.loss_seq) p.loss_seq[b] = total;
@@ -234,36 +281,28 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         return;
     }
 
-    // ---- sampler epilogue ----
-    // argmax: the first chunk whose raw maximum is the row maximum, then the first id in it.
+    // ---- sampler epilogue
+    // argmax chunk: the first chunk whose raw maximum is the row maximum.
     int jm = 0x7fffffff;
-    for (int32_t j = tid; j < nch; j += kPassThreads)
-        if (ld_cg_f4(rec + j).x == m_raw) {
-            jm = j;
-            break;
-        }
+#pragma unroll
+    for (int k = 3; k >= 0; --k)
+        if (r[k].x == m_raw) jm = 4 * tid + k;
+    for (int32_t q = tid + kPassThreads; 4 * q < nch && jm == 0x7fffffff; q += kPassThreads) {
+        float4 f[4];
+        far_quad(q, f);
+#pragma unroll
+        for (int k = 3; k >= 0; --k)
+            if (f[k].x == m_raw) jm = 4 * q + k;
+    }
     jm = block_min_int<kPassWarps>(jm, sh.i);
     if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
-    int am = 0x7fffffff;
-    {
-        const int32_t lo = jm * kChunk, hi = min(lo + kChunk, p.V);
-        for (int32_t v = lo + tid; v < hi; v += kPassThreads)
-            if (fmaxf(load_logit(rowp, v, kBf16), nbig) == m_raw) {
-                am = v;
-                break;
-            }
-    }
-    am = block_min_int<kPassWarps>(am, sh.i);
-    if (am >= p.V) am = jm * kChunk;
 
-    int32_t x0;
-    if (p.mode == DG_X0_GREEDY) {
-        x0 = am;
-    } else {
-        // Level 1: chunk scores lse_c + G_c; thread q scores chunks 4q .. 4q+3 from one Philox call.
+    // Level 1: chunk scores lse_c + G_c, four chunks per Philox call.
+    int32_t bj = jm;
+    if (p.mode != DG_X0_GREEDY) {
         float bs = -INFINITY;
-        int bj = 0x7fffffff;
-        for (int32_t q = tid; 4 * q < nch; q += kPassThreads) {
+        int bjl = 0x7fffffff;
+        auto score_quad = [&](int32_t q, const float4 (&f)[4]) {
             const uint4 w = philox4x32_10(
                 make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
                 p.key1);
@@ -271,40 +310,66 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             for (int k = 0; k < 4; ++k) {
                 const int32_t j = 4 * q + k;
                 if (j < nch) {
-                    const float4 r = ld_cg_f4(rec + j);
-                    const float sc = (r.x * inv_tau + logf(r.y)) + gumbel_from_word(word_of(w, k));
+                    const float sc = (f[k].x * inv_tau + logf(f[k].y)) + gumbel_from_word(word_of(w, k));
                     if (sc > bs) {
                         bs = sc;
-                        bj = j;
+                        bjl = j;
                     }
                 }
             }
+        };
+        if (4 * tid < nch) score_quad(tid, r);
+        for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
+            float4 f[4];
+            far_quad(q, f);
+            score_quad(q, f);
         }
-        block_argmax<kPassWarps>(bs, bj, sh.f, sh.i);
-        if (bj >= nch) bj = jm;  // NaN scores only
-        // Level 2: the ids of the winning chunk; thread q < 128 takes ids lo + 4q .. lo + 4q + 3.
-        const int32_t lo = bj * kChunk, hi = min(lo + kChunk, p.V);
+        block_argmax<kPassWarps>(bs, bjl, sh.f, sh.i);
+        bj = bjl < nch ? bjl : jm;  // NaN scores only
+    }
+
+    // One round trip for both re-read chunks: ids lo + 4 tid .. lo + 4 tid + 3 of each.
+    const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
+    const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
+    float av[4], gv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int32_t va = alo + 4 * tid + k, vg = glo + 4 * tid + k;
+        av[k] = va < ahi ? fmaxf(load_logit(rowp, va, kBf16), nbig) : -INFINITY;
+        gv[k] = vg < ghi ? fmaxf(load_logit(rowp, vg, kBf16), nbig) : -INFINITY;
+    }
+    int am = 0x7fffffff;
+#pragma unroll
+    for (int k = 3; k >= 0; --k)
+        if (alo + 4 * tid + k < ahi && av[k] == m_raw) am = alo + 4 * tid + k;
+    am = block_min_int<kPassWarps>(am, sh.i);
+    if (am >= p.V) am = jm * kChunk;
+
+    int32_t x0;
+    if (p.mode == DG_X0_GREEDY) {
+        x0 = am;
+    } else {
+        // Level 2: argmax of l'_v + G_v over the winning chunk, four ids per Philox call.
         float bs2 = -INFINITY;
         int bv = 0x7fffffff;
-        const int32_t vg = lo + 4 * tid;
-        if (tid < kChunk / 4 && vg < hi) {
+        const int32_t vg0 = glo + 4 * tid;
+        if (vg0 < ghi) {
             const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(vg) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
+                make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
                 p.key0, p.key1);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int32_t v = vg + k;
-                if (v < hi) {
-                    const float sc = fmaxf(load_logit(rowp, v, kBf16), nbig) * inv_tau + gumbel_from_word(word_of(w, k));
+                if (vg0 + k < ghi) {
+                    const float sc = gv[k] * inv_tau + gumbel_from_word(word_of(w, k));
                     if (sc > bs2) {
                         bs2 = sc;
-                        bv = v;
+                        bv = vg0 + k;
                     }
                 }
             }
         }
         block_argmax<kPassWarps>(bs2, bv, sh.f, sh.i);
-        x0 = (bv >= lo && bv < hi) ? bv : am;
+        x0 = (bv >= glo && bv < ghi) ? bv : am;
     }
 
     if (tid == 0) {
@@ -343,7 +408,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 }
 
 template <bool kBf16, int kKind>
-__global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_constant__ PassParams p) {
+__global__ void __launch_bounds__(kPassThreads, 8) logits_pass_kernel(const __grid_constant__ PassParams p) {
     __shared__ MergeShared sh;
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;
