@@ -408,7 +408,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 }
 
 template <bool kBf16, int kKind>
-__global__ void __launch_bounds__(kPassThreads, 8) logits_pass_kernel(const __grid_constant__ PassParams p) {
+__global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_constant__ PassParams p) {
     __shared__ MergeShared sh;
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;
