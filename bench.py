@@ -64,6 +64,19 @@ def dist_env():
     return rank, world, local
 
 
+def whole_job_rate(local_ms: float, units_per_rank: int, world: int, device="cpu"):
+    """Max over ranks of the per-rank device time (ms) and the whole-job rate: every rank
+    processed `units_per_rank` units, so the job did world * units_per_rank in the slowest
+    rank's time.  Collective only when world > 1 (the data path itself exchanges nothing)."""
+    import torch
+    ms = float(local_ms)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, world * units_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
@@ -235,11 +248,7 @@ def run_ours(args, rank, world, local):
     k2_us = [ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) * 1e3 for k in range(K)]
     dev_err = dg.dg_device_error()
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    steps_per_s = world * K / (total_ms / 1e3)
+    total_ms, steps_per_s = whole_job_rate(total_ms, K, world, dev)
 
     # ---- roofline of the dominant kernel (the contraction) and of the logits pass
     k1_mean = statistics.mean(k1_us)
@@ -389,12 +398,8 @@ def bench_e2e(dg, W, cfg, dev, E, args, world, barrier):
             one(k)
         e1.record(stream)
     stream.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * steps / (ms / 1e3), 2), "unit": "steps/s",
+    ms, rate = whole_job_rate(e0.elapsed_time(e1), steps, world, dev)
+    return {"value": round(rate, 2), "unit": "steps/s",
             "h2d_bytes_per_step": host_logits.numel() * host_logits.element_size(),
             "d2h_bytes_per_step": host_x.numel() * 4 + host_z.numel() * 2, "steps": steps}
 

@@ -51,6 +51,9 @@ def lib() -> ctypes.CDLL:
         L.dg_version.restype = ctypes.c_char_p
         L.dg_launch_count.restype = _u64
         L.dg_device_error.argtypes = [_p]
+        L.dg_test_bounded_wait.argtypes = [_u32, _p]
+        L.dg_test_selfcond_stall.argtypes = [_p, _int, _i64, _i32, _i32, _i32, _p, _p, _p, _int, _i32, _p, _p, _sz,
+                                             _p, _i32, _u32]
         L.dg_sampler_step_workspace_size.argtypes = [_i32, _i32]
         L.dg_sampler_step_workspace_size.restype = _sz
         L.dg_sampler_step.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32, _int,

@@ -348,9 +348,13 @@ size_t dg_selfcond_workspace_size(int32_t rows, int32_t V, int32_t d, int logits
     return n;
 }
 
-int dg_selfcond(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
-                const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d, void* z,
-                void* workspace, size_t workspace_bytes, dg_stream_t stream) {
+}  // extern "C"
+
+namespace {
+int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
+                  const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d, void* z,
+                  void* workspace, size_t workspace_bytes, dg_stream_t stream, int32_t fault_block,
+                  long long wait_limit) {
     g_last_error.clear();
     int rc;
     if ((rc = check_logits(logits, logits_dtype, ld, V)) != DG_OK) return rc;
@@ -418,9 +422,44 @@ int dg_selfcond(const void* logits, int logits_dtype, int64_t ld, int32_t B, int
     sp.d = d;
     // partial sums and tile tickets live at the end of the workspace
     sp.partial = reinterpret_cast<float*>(wp);
+    sp.wait_limit = wait_limit;
+    sp.fault_block = fault_block;
     const cudaError_t e = launch_selfcond(sp, s);
     if (e != cudaSuccess) return cuda_fail(e, "self-conditioning launch");
     return DG_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int dg_selfcond(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
+                const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d, void* z,
+                void* workspace, size_t workspace_bytes, dg_stream_t stream) {
+    return selfcond_impl(logits, logits_dtype, ld, B, C, V, inv_tau, lse, E, embed_dtype, d, z, workspace,
+                         workspace_bytes, stream, -1, 0);
+}
+
+int dg_test_bounded_wait(uint32_t limit_cycles, dg_stream_t stream) {
+    g_last_error.clear();
+    if (limit_cycles == 0) return fail(DG_ERR_INVALID_ARG, "limit_cycles must be > 0");
+    int rc;
+    if ((rc = check_device()) != DG_OK) return rc;
+    const cudaError_t e = launch_bounded_wait_test(static_cast<long long>(limit_cycles),
+                                                   reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "bounded-wait test launch");
+    return DG_OK;
+}
+
+int dg_test_selfcond_stall(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
+                           const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d,
+                           void* z, void* workspace, size_t workspace_bytes, dg_stream_t stream,
+                           int32_t stalled_block, uint32_t limit_cycles) {
+    if (stalled_block < 0 || limit_cycles == 0) {
+        g_last_error = "stalled_block must be >= 0 and limit_cycles > 0";
+        return DG_ERR_INVALID_ARG;
+    }
+    return selfcond_impl(logits, logits_dtype, ld, B, C, V, inv_tau, lse, E, embed_dtype, d, z, workspace,
+                         workspace_bytes, stream, stalled_block, static_cast<long long>(limit_cycles));
 }
 
 }  // extern "C"

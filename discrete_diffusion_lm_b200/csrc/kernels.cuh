@@ -79,12 +79,16 @@ struct SelfcondParams {
     uint16_t* z;         // bf16 [R, d]
     float* partial;      // fp32 [splits, R, d] (when the vocabulary is split)
     int32_t R, C, V, d;
+    long long wait_limit;  // cycles before a stalled wait aborts the CTA (0: the library default)
+    int32_t fault_block;   // test hook: never issue the E copy of this 32-id block (-1: none)
     float inv_tau[DG_MAX_CANVASES];
 };
 
 size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d);
 cudaError_t launch_selfcond(const SelfcondParams& p, cudaStream_t s);
 cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s);
+// One thread waits on a barrier nothing arrives on; the bounded wait must give up (test).
+cudaError_t launch_bounded_wait_test(long long limit_cycles, cudaStream_t s);
 // Reads (synchronously) and clears the error word set by a kernel whose bounded wait expired.
 cudaError_t read_and_clear_device_error(int* out);
 

@@ -49,6 +49,8 @@ struct alignas(64) KernelParams {
     float* partial;
     int32_t R, C, V, d;
     int32_t n_tiles, splits, total_kb;
+    long long wait_limit;  // cycles a wait may last before the CTA aborts
+    int32_t fault_block;   // test hook: the E copy of this 32-id block is never issued (-1: none)
     float inv_tau[DG_MAX_CANVASES];
 };
 
@@ -91,16 +93,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Per-CTA wait control in shared memory: the abort flag every wait watches, and the wait limit.
+struct WaitCtl {
+    int abort;
+    int pad;
+    long long limit;  // cycles
+};
+__device__ __forceinline__ bool aborted(const WaitCtl* c) { return *reinterpret_cast<const volatile int*>(&c->abort) != 0; }
+
 // Wait for the phase with the given parity to complete.  Gives up (returning false) when another
-// thread of the CTA has aborted or after kWaitLimitCycles, recording the expiry.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// thread of the CTA has aborted or after ctl->limit cycles, recording the expiry.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort_flag = 1;
+        if (aborted(ctl)) return false;
+        if (clock64() - t0 > ctl->limit) {
+            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
             atomicExch(&g_device_error, 1);
             return false;
         }
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
     uint64_t* empty = pready + kStages;
     uint64_t* accum = empty + kStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    WaitCtl* wc = reinterpret_cast<WaitCtl*>(tmem_slot + 2);
 
     int bid = blockIdx.x;
     const int split = bid % p.splits;
@@ -233,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
-        *abort_flag = 0;
+        wc->abort = 0;
+        wc->limit = p.wait_limit;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -254,25 +265,28 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
+                if (!mbar_wait(&empty[s], ph ^ 1, wc)) break;
                 uint8_t* st = smem + s * G::kStageBytes;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
                 tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mt * kTileM, &lfull[s]);
-                mbar_arrive_expect_tx(&efull[s], G::kEBytes);
+                if (kb0 + i * kstride != p.fault_block) {
+                    mbar_arrive_expect_tx(&efull[s], G::kEBytes);
 #pragma unroll
-                for (int b = 0; b < kNT / 64; ++b)
-                    tma_load_2d(st + b * (64 * kKBlock * 2), &p.tm_E, nt * kNT + 64 * b, k0, &efull[s]);
+                    for (int b = 0; b < kNT / 64; ++b)
+                        tma_load_2d(st + b * (64 * kKBlock * 2), &p.tm_E, nt * kNT + 64 * b, k0, &efull[s]);
+                }
                 issued = i + 1;
             }
-            if (*abort_flag) {
+            if (aborted(wc)) {
                 // let the copies already issued land before the CTA's shared memory goes away
+                const long long t0 = clock64();  // one deadline for the whole drain
                 for (int i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i) {
                     const int s = i % kStages;
                     const uint32_t ph = (i / kStages) & 1;
-                    const long long t0 = clock64();
-                    while (!(mbar_try_wait(&lfull[s], ph) && mbar_try_wait(&efull[s], ph)) &&
-                           clock64() - t0 < kWaitLimitCycles) {
+                    const bool e_issued = kb0 + i * kstride != p.fault_block;
+                    while (!(mbar_try_wait(&lfull[s], ph) && (!e_issued || mbar_try_wait(&efull[s], ph))) &&
+                           clock64() - t0 < wc->limit) {
                     }
                 }
             }
@@ -285,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_wait(&efull[s], ph, abort_flag)) break;
-                if (!mbar_wait(&pready[s], ph, abort_flag)) break;
+                if (!mbar_wait(&efull[s], ph, wc)) break;
+                if (!mbar_wait(&pready[s], ph, wc)) break;
                 tcgen05_after_sync();
                 uint8_t* st = smem + s * G::kStageBytes;
                 const uint32_t a_base = smem_u32(st + G::kEBytes + (kBf16 ? 0 : G::kLBytes));
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         for (int i = group; i < nkb; i += 2) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
-            const bool ok = mbar_wait(&lfull[s], ph, abort_flag);
+            const bool ok = mbar_wait(&lfull[s], ph, wc);
             uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
             if (!ok) {
             } else if (kBf16) {
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             if (softmax_group_sync_or(group, !ok)) break;
             if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, abort_flag))) {
+        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, wc))) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
             for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
@@ -458,14 +472,14 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 // Bounded wait with cluster-scope acquire (arrivals may come from the other CTA of the pair).
-__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort_flag = 1;
+        if (aborted(ctl)) return false;
+        if (clock64() - t0 > ctl->limit) {
+            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
             atomicExch(&g_device_error, 1);
             return false;
         }
@@ -510,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     uint64_t* pready = lempty + kLS;                   // leader: both CTAs' p; peer: own p (forwarded)
     uint64_t* accum = pready + kLS;                    // own accumulator final
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    WaitCtl* wc = reinterpret_cast<WaitCtl*>(tmem_slot + 2);
 
     const uint32_t rank = cluster_rank();
     int bid = blockIdx.x >> 1;  // pair index
@@ -537,7 +551,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             mbar_init(&pready[s], rank == 0 ? 2 : 1);
         }
         mbar_init(accum, 1);
-        *abort_flag = 0;
+        wc->abort = 0;
+        wc->limit = p.wait_limit;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -559,8 +574,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kES;
                 const uint32_t ph = (i / kES) & 1;
-                if (!mbar_wait(&eempty[s], ph ^ 1, abort_flag)) break;
+                if (!mbar_wait(&eempty[s], ph ^ 1, wc)) break;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
+                issued = i + 1;
+                if (kb0 + i * kstride == p.fault_block) continue;
                 if (rank == 0) mbar_arrive_expect_tx(&efull[s], 2 * G::kEBytes);
                 uint8_t* dst = ering + s * G::kEBytes;
 #pragma unroll
@@ -571,13 +588,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         tma_load_2d_pair(dst + (nh * G::kBoxesPerHalf + j) * (64 * kKBlock * 2), &p.tm_E, col, k0,
                                          leader_efull0 + s * 8);
                     }
-                issued = i + 1;
             }
-            if (*abort_flag && rank == 0) {
+            if (aborted(wc) && rank == 0) {
                 // both halves of the last stages land on the leader's barriers: wait for them (bounded)
+                const long long t0 = clock64();  // one deadline for the whole drain
                 for (int i = issued - kES > 0 ? issued - kES : 0; i < issued; ++i) {
-                    const long long t0 = clock64();
-                    while (!mbar_try_wait(&efull[i % kES], (i / kES) & 1) && clock64() - t0 < kWaitLimitCycles) {
+                    if (kb0 + i * kstride == p.fault_block) continue;
+                    while (!mbar_try_wait(&efull[i % kES], (i / kES) & 1) && clock64() - t0 < wc->limit) {
                     }
                 }
             }
@@ -589,17 +606,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kLS;
                 const uint32_t ph = (i / kLS) & 1;
-                if (!mbar_wait(&lempty[s], ph ^ 1, abort_flag)) break;
+                if (!mbar_wait(&lempty[s], ph ^ 1, wc)) break;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
                 tma_load_2d(lring + s * G::kLStageBytes, &p.tm_logits, k0,
                             mp * 2 * kTileM + static_cast<int>(rank) * kTileM, &lfull[s]);
                 issued = i + 1;
             }
-            if (*abort_flag) {
+            if (aborted(wc)) {
+                const long long t0 = clock64();  // one deadline for the whole drain
                 for (int i = issued - kLS > 0 ? issued - kLS : 0; i < issued; ++i) {
-                    const long long t0 = clock64();
-                    while (!mbar_try_wait(&lfull[i % kLS], (i / kLS) & 1) && clock64() - t0 < kWaitLimitCycles) {
+                    while (!mbar_try_wait(&lfull[i % kLS], (i / kLS) & 1) && clock64() - t0 < wc->limit) {
                     }
                 }
             }
@@ -611,7 +628,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t leader_pready0 = map_to_rank(smem_u32(&pready[0]), 0);
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kLS;
-                if (!mbar_wait(&pready[s], (i / kLS) & 1, abort_flag)) break;
+                if (!mbar_wait(&pready[s], (i / kLS) & 1, wc)) break;
                 mbar_arrive_remote(leader_pready0 + s * 8);
             }
         }
@@ -625,8 +642,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t lempty_peer = map_to_rank(smem_u32(&lempty[0]), 1);
             for (int i = 0; i < nkb; ++i) {
                 const int es = i % kES, ls = i % kLS;
-                if (!mbar_wait(&efull[es], (i / kES) & 1, abort_flag)) break;
-                if (!mbar_wait(&pready[ls], (i / kLS) & 1, abort_flag)) break;
+                if (!mbar_wait(&efull[es], (i / kES) & 1, wc)) break;
+                if (!mbar_wait(&pready[ls], (i / kLS) & 1, wc)) break;
                 tcgen05_after_sync();
                 const uint32_t a_base = smem_u32(lring + ls * G::kLStageBytes + (kBf16 ? 0 : G::kLBytes));
                 const uint32_t b_base = smem_u32(ering + es * G::kEBytes);
@@ -662,7 +679,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int leader_thread = (kFirstSoftmaxWarp + 4 * group) * 32;
         for (int i = group; i < nkb; i += 2) {
             const int s = i % kLS;
-            const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, abort_flag);
+            const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, wc);
             uint8_t* lt = lring + s * G::kLStageBytes;
             if (!ok) {
             } else if (kBf16) {
@@ -693,7 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (softmax_group_sync_or(group, !ok)) break;
             if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, abort_flag))) {
+        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, wc))) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
             for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
@@ -734,6 +751,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     if (warp == 1)
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(static_cast<uint32_t>(kNT))
                      : "memory");
+}
+
+// Test of the bounded wait itself: one thread waits on a barrier that nothing will ever arrive on.
+// The wait gives up after `limit` cycles, records device error 1 and the kernel returns normally.
+__global__ void bounded_wait_test_kernel(long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ WaitCtl wc;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        wc.abort = 0;
+        wc.limit = limit;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &wc);
+    __syncthreads();
 }
 
 // z[i] = bf16(sum_s partial[s][i]) in a fixed order (deterministic).
@@ -898,6 +931,8 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     kp.n_tiles = pl.n_tiles;
     kp.splits = splits;
     kp.total_kb = pl.total_kb;
+    kp.wait_limit = sp.wait_limit > 0 ? sp.wait_limit : kWaitLimitCycles;
+    kp.fault_block = sp.fault_block;
     std::memcpy(kp.inv_tau, sp.inv_tau, sizeof(kp.inv_tau));
     const int grid = pl.ctas;
 #define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st)
@@ -938,6 +973,12 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
 cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s) {
     const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 8LL * num_sms()));
     convert_f32_bf16_kernel<<<blocks, 256, 0, s>>>(in, out, n);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bounded_wait_test(long long limit_cycles, cudaStream_t st) {
+    bounded_wait_test_kernel<<<1, 32, 0, st>>>(limit_cycles);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -175,6 +175,28 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
                  size_t workspace_bytes, dg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Failure-detection test hooks (the pages have no counterpart).  Every wait */
+/* inside the library's kernels is bounded; these entry points make a wait  */
+/* run out on purpose -- without any fault, trap or endless loop -- so that */
+/* tests can check that the kernel gives up, reports through                */
+/* dg_device_error() (code 1) and leaves the device usable.                 */
+/* dg_test_bounded_wait: one thread waits on a barrier nothing arrives on;  */
+/*   the wait gives up after limit_cycles (> 0) SM clock cycles.             */
+/* dg_test_selfcond_stall: dg_selfcond with the copy of one 32-id block of  */
+/*   E never issued (stalled_block >= 0, in [0, ceil(V/32)) to take effect) */
+/*   and every wait limited to limit_cycles: the CTAs that need the block   */
+/*   abort, drain their in-flight copies, free their tensor memory and      */
+/*   return.  z is then incomplete.  Same arguments as dg_selfcond otherwise.*/
+/* ------------------------------------------------------------------------ */
+int dg_test_bounded_wait(uint32_t limit_cycles, dg_stream_t stream);
+
+int dg_test_selfcond_stall(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C,
+                           int32_t V, const float* inv_tau, const float* lse, const void* E,
+                           int embed_dtype, int32_t d, void* z, void* workspace,
+                           size_t workspace_bytes, dg_stream_t stream, int32_t stalled_block,
+                           uint32_t limit_cycles);
+
+/* ------------------------------------------------------------------------ */
 /* Allocation-free sampler step.  The pages have no counterpart: this entry  */
 /* point exists for callers that cannot allocate device memory where they   */
 /* sample (a serving loop that must not call cudaMalloc, which can stall the */
