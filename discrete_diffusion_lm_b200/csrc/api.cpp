@@ -344,7 +344,7 @@ size_t dg_selfcond_workspace_size(int32_t rows, int32_t V, int32_t d, int logits
     size_t n = 0;
     if (!have_lse) n += align_up(static_cast<size_t>(rows) * 4, 256) + align_up(pass_ws_bytes(rows, V, 0), 256);
     if (embed_dtype == DG_F32) n += align_up(static_cast<size_t>(V) * d * 2, 256);
-    n += selfcond_partial_bytes(rows, V, d);
+    n += selfcond_partial_bytes(rows, V, d, logits_dtype == DG_BF16);
     return n;
 }
 

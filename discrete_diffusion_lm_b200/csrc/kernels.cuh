@@ -84,7 +84,7 @@ struct SelfcondParams {
     float inv_tau[DG_MAX_CANVASES];
 };
 
-size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d);
+size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16);
 cudaError_t launch_selfcond(const SelfcondParams& p, cudaStream_t s);
 cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s);
 // One thread waits on a barrier nothing arrives on; the bounded wait must give up (test).

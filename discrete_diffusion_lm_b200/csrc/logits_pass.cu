@@ -434,9 +434,11 @@ __global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_
         const int32_t c = 4 * gi + (lane >> 3);
         if ((lane & 7) == 0 && c < p.n_chunks) rec[c] = make_float4(cs.m_raw, cs.S, cs.T, 0.f);
     }
-    __threadfence();
+    // The barrier orders every warp's record stores before thread 0's fence, and the fence is
+    // cumulative: one fence makes the whole CTA's records visible before its ticket increment.
     __syncthreads();
     if (threadIdx.x == 0) {
+        __threadfence();
         const unsigned prev = atomicAdd(&p.row_ticket[row], 1u);
         sh.flag = prev == static_cast<unsigned>(p.segs - 1);
     }

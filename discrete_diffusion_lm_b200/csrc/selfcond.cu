@@ -5,12 +5,12 @@
 // expected embedding p0 E is the dense contraction computed here (the trained FFW is not).
 //
 // One CTA computes a 128-row x kNT-column tile of z over a contiguous range of the vocabulary
-// (split-K).  Per stage of kKBlock = 32 ids:
-//   * a producer thread TMA-loads the E tile [32 ids x kNT] (MN-major, 128-byte swizzle, boxes of
-//     64 columns) and the logits tile [128 rows x 32 ids] (64-byte swizzle for bf16);
+// (split-K).  Per stage of kKBlock = 64 ids:
+//   * a producer thread TMA-loads the E tile [64 ids x kNT] (MN-major, 128-byte swizzle, boxes of
+//     64 columns) and the logits tile [128 rows x 64 ids] (128-byte swizzle);
 //   * four softmax warps turn each thread's logits row into p = exp2(l * a - lse * log2 e), i.e.
 //     softmax(l') with the row's log-sum-exp from the logits pass, round it to bf16 and write it
-//     back in the K-major 64-byte-swizzled layout the tensor core reads as operand A;
+//     back in the K-major 128-byte-swizzled layout the tensor core reads as operand A;
 //   * one thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into a TMEM accumulator of
 //     128 lanes x kNT columns and commits the stage back to the producer.
 // Because lse is known, p is final when it is formed: no running-max rescale of the accumulator is
@@ -34,7 +34,7 @@ __device__ int g_device_error = 0;  // set by a kernel whose bounded wait expire
 
 namespace {
 
-constexpr int kKBlock = 32;  // vocabulary ids per pipeline stage
+constexpr int kKBlock = 64;  // vocabulary ids per pipeline stage
 constexpr int kTileM = 128;  // rows per CTA = TMEM lanes
 constexpr int kNumSoftmaxWarps = 8;  // two groups of four; group g converts the stages i with i % 2 == g
 constexpr int kGroupThreads = 128;
@@ -157,7 +157,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     d |= static_cast<uint64_t>(layout & 7u) << 61;
     return d;
 }
-constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+constexpr uint32_t kLayoutSw128 = 2;
 
 // Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, A K-major, B MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
@@ -207,6 +207,46 @@ __device__ __forceinline__ uint4 softmax_chunk_bf16(uint4 c, float a, float nb) 
 }
 __device__ __forceinline__ uint32_t softmax_pair_f32(uint32_t x, uint32_t y, float a, float nb) {
     return pack_bf16x2(ex2_approx(fmaf(__uint_as_float(x), a, nb)), ex2_approx(fmaf(__uint_as_float(y), a, nb)));
+}
+
+// Turn one logits row of the stage tile into p = exp2(l * a + nb) as the bf16 K-major A operand.
+// Rows are 128 bytes with the 128-byte swizzle: 16-byte chunk j of row r sits at j ^ (r & 7).
+// bf16 logits are converted in place; fp32 logits arrive as two [128 x 32] sub-tiles and p goes
+// to the separate bf16 tile `pt`.
+template <bool kBf16>
+__device__ __forceinline__ void softmax_row(uint8_t* lt, uint8_t* pt, int row, float a, float nb) {
+    const int sw = row & 7;
+    if (kBf16) {
+        uint8_t* rb = lt + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint4* q = reinterpret_cast<uint4*>(rb + ((j ^ sw) << 4));
+            *q = softmax_chunk_bf16(*q, a, nb);
+        }
+    } else {
+        uint8_t* pb = pt + row * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint8_t* rb = lt + (q >> 2) * (kTileM * 128) + row * 128;
+            const int c = 2 * (q & 3);
+            const uint4 c0 = *reinterpret_cast<const uint4*>(rb + ((c ^ sw) << 4));
+            const uint4 c1 = *reinterpret_cast<const uint4*>(rb + (((c + 1) ^ sw) << 4));
+            uint4 o;
+            o.x = softmax_pair_f32(c0.x, c0.y, a, nb);
+            o.y = softmax_pair_f32(c0.z, c0.w, a, nb);
+            o.z = softmax_pair_f32(c1.x, c1.y, a, nb);
+            o.w = softmax_pair_f32(c1.z, c1.w, a, nb);
+            *reinterpret_cast<uint4*>(pb + ((q ^ sw) << 4)) = o;
+        }
+    }
+}
+
+// Logits tile copy of one stage: one box of 64 bf16 ids, or two boxes of 32 fp32 ids.
+template <bool kBf16>
+__device__ __forceinline__ void load_logits_tile(uint8_t* dst, const CUtensorMap* tm, int32_t k0, int32_t row0,
+                                                 uint64_t* bar) {
+    tma_load_2d(dst, tm, k0, row0, bar);
+    if (!kBf16) tma_load_2d(dst + kTileM * 128, tm, k0 + 32, row0, bar);
 }
 
 template <bool kBf16, int kNT>
@@ -269,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                 uint8_t* st = smem + s * G::kStageBytes;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
-                tma_load_2d(st + G::kEBytes, &p.tm_logits, k0, mt * kTileM, &lfull[s]);
+                load_logits_tile<kBf16>(st + G::kEBytes, &p.tm_logits, k0, mt * kTileM, &lfull[s]);
                 if (kb0 + i * kstride != p.fault_block) {
                     mbar_arrive_expect_tx(&efull[s], G::kEBytes);
 #pragma unroll
@@ -307,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                 const uint32_t b_base = smem_u32(st);
 #pragma unroll
                 for (int ks = 0; ks < kKBlock / 16; ++ks) {
-                    // A: 128 rows x 16 ids, K-major, rows of 64 bytes, 8-row atoms of 512 bytes
-                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 512, kLayoutSw64);
+                    // A: 128 rows x 16 ids, K-major, rows of 128 bytes, 8-row atoms of 1 KB
+                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 1024, kLayoutSw128);
 #pragma unroll
                     for (int nh = 0; nh < kNT / kMmaN; ++nh) {
                         // B: 16 ids x kMmaN columns, MN-major, 64-column boxes 4 KB apart, 8-id atoms of 1 KB
@@ -337,33 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             const uint32_t ph = (i / kStages) & 1;
             const bool ok = mbar_wait(&lfull[s], ph, wc);
             uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
-            if (!ok) {
-            } else if (kBf16) {
-                // row of 32 bf16 = 64 bytes; 16-byte chunk j stored at j ^ ((row >> 1) & 3)
-                uint8_t* rb = lt + row * 64;
-                const int sw = (row >> 1) & 3;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4* q = reinterpret_cast<uint4*>(rb + ((j ^ sw) << 4));
-                    *q = softmax_chunk_bf16(*q, a, nb);
-                }
-            } else {
-                // fp32 row of 32 ids = 128 bytes, chunk j at j ^ (row & 7); p goes to the bf16 tile
-                const uint8_t* rb = lt + row * 128;
-                uint8_t* pb = lt + G::kLBytes + row * 64;
-                const int sw8 = row & 7, sw4 = (row >> 1) & 3;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 c0 = *reinterpret_cast<const uint4*>(rb + (((2 * q) ^ sw8) << 4));
-                    const uint4 c1 = *reinterpret_cast<const uint4*>(rb + (((2 * q + 1) ^ sw8) << 4));
-                    uint4 o;
-                    o.x = softmax_pair_f32(c0.x, c0.y, a, nb);
-                    o.y = softmax_pair_f32(c0.z, c0.w, a, nb);
-                    o.z = softmax_pair_f32(c1.x, c1.y, a, nb);
-                    o.w = softmax_pair_f32(c1.z, c1.w, a, nb);
-                    *reinterpret_cast<uint4*>(pb + ((q ^ sw4) << 4)) = o;
-                }
-            }
+            if (ok) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
             fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
             if (softmax_group_sync_or(group, !ok)) break;
             if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);
@@ -609,8 +623,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 if (!mbar_wait(&lempty[s], ph ^ 1, wc)) break;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
                 mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
-                tma_load_2d(lring + s * G::kLStageBytes, &p.tm_logits, k0,
-                            mp * 2 * kTileM + static_cast<int>(rank) * kTileM, &lfull[s]);
+                load_logits_tile<kBf16>(lring + s * G::kLStageBytes, &p.tm_logits, k0,
+                                        mp * 2 * kTileM + static_cast<int>(rank) * kTileM, &lfull[s]);
                 issued = i + 1;
             }
             if (aborted(wc)) {
@@ -649,7 +663,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const uint32_t b_base = smem_u32(ering + es * G::kEBytes);
 #pragma unroll
                 for (int ks = 0; ks < kKBlock / 16; ++ks) {
-                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 512, kLayoutSw64);
+                    const uint64_t adesc = smem_desc(a_base + ks * 32, 16, 1024, kLayoutSw128);
 #pragma unroll
                     for (int nh = 0; nh < kNT / G::kMmaN; ++nh) {
                         const uint64_t bdesc = smem_desc(
@@ -681,31 +695,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const int s = i % kLS;
             const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, wc);
             uint8_t* lt = lring + s * G::kLStageBytes;
-            if (!ok) {
-            } else if (kBf16) {
-                uint8_t* rb = lt + row * 64;
-                const int sw = (row >> 1) & 3;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4* q = reinterpret_cast<uint4*>(rb + ((j ^ sw) << 4));
-                    *q = softmax_chunk_bf16(*q, a, nb);
-                }
-            } else {
-                const uint8_t* rb = lt + row * 128;
-                uint8_t* pb = lt + G::kLBytes + row * 64;
-                const int sw8 = row & 7, sw4 = (row >> 1) & 3;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 c0 = *reinterpret_cast<const uint4*>(rb + (((2 * q) ^ sw8) << 4));
-                    const uint4 c1 = *reinterpret_cast<const uint4*>(rb + (((2 * q + 1) ^ sw8) << 4));
-                    uint4 o;
-                    o.x = softmax_pair_f32(c0.x, c0.y, a, nb);
-                    o.y = softmax_pair_f32(c0.z, c0.w, a, nb);
-                    o.z = softmax_pair_f32(c1.x, c1.y, a, nb);
-                    o.w = softmax_pair_f32(c1.z, c1.w, a, nb);
-                    *reinterpret_cast<uint4*>(pb + ((q ^ sw4) << 4)) = o;
-                }
-            }
+            if (ok) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
             fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
             if (softmax_group_sync_or(group, !ok)) break;
             if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
@@ -825,7 +815,12 @@ cudaError_t encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base,
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int pick_ntile(int d) { return d % 512 == 0 ? 512 : d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64; }
+// Column tile: 512 when d allows; fp32 logits (small test workloads) stage twice the bytes per
+// tile and use at most 256 columns so that the pipeline keeps its depth.
+int pick_ntile(int d, bool logits_bf16) {
+    const int nt = d % 512 == 0 ? 512 : d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
+    return logits_bf16 ? nt : (nt > 256 ? 256 : nt);
+}
 
 int num_sms() {
     static std::atomic<int> cached{0};
@@ -851,9 +846,9 @@ struct Plan {
     int ctas;
 };
 
-Plan plan(int R, int V, int d) {
+Plan plan(int R, int V, int d, bool logits_bf16) {
     Plan pl;
-    const int nt = pick_ntile(d);
+    const int nt = pick_ntile(d, logits_bf16);
     pl.pair = R > kTileM && nt >= 128;
     pl.m_tiles = pl.pair ? (R + 2 * kTileM - 1) / (2 * kTileM) : (R + kTileM - 1) / kTileM;
     pl.n_tiles = d / nt;
@@ -898,25 +893,25 @@ cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st
 
 }  // namespace
 
-size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d) {
+size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16) {
     if (R < 1 || V < 1 || d < 64) return 0;
-    const Plan pl = plan(R, V, d);
+    const Plan pl = plan(R, V, d, logits_bf16);
     return pl.splits > 1 ? static_cast<size_t>(pl.splits) * R * d * sizeof(float) : 0;
 }
 
 cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     static thread_local KernelParams kp;
     std::memset(&kp, 0, sizeof(kp));
-    const Plan pl = plan(sp.R, sp.V, sp.d);
+    const Plan pl = plan(sp.R, sp.V, sp.d, sp.logits_bf16 != 0);
     const int splits = pl.splits;
-    const int nt = pick_ntile(sp.d);
+    const int nt = pick_ntile(sp.d, sp.logits_bf16 != 0);
     cudaError_t e;
     if (sp.logits_bf16)
         e = encode_2d(&kp.tm_logits, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.logits, sp.V, sp.R,
-                      static_cast<uint64_t>(sp.ld) * 2, kKBlock, kTileM, CU_TENSOR_MAP_SWIZZLE_64B);
+                      static_cast<uint64_t>(sp.ld) * 2, kKBlock, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
     else
         e = encode_2d(&kp.tm_logits, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.logits, sp.V, sp.R,
-                      static_cast<uint64_t>(sp.ld) * 4, kKBlock, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
+                      static_cast<uint64_t>(sp.ld) * 4, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     e = encode_2d(&kp.tm_E, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.E, sp.d, sp.V, static_cast<uint64_t>(sp.d) * 2, 64,
                   kKBlock, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -943,8 +938,7 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
             else if (nt == 256) DG_PC(true, 256);
             else DG_PC(true, 128);
         } else {
-            if (nt == 512) DG_PC(false, 512);
-            else if (nt == 256) DG_PC(false, 256);
+            if (nt == 256) DG_PC(false, 256);
             else DG_PC(false, 128);
         }
     } else if (sp.logits_bf16) {
@@ -953,8 +947,7 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
         else if (nt == 128) DG_SC(true, 128);
         else DG_SC(true, 64);
     } else {
-        if (nt == 512) DG_SC(false, 512);
-        else if (nt == 256) DG_SC(false, 256);
+        if (nt == 256) DG_SC(false, 256);
         else if (nt == 128) DG_SC(false, 128);
         else DG_SC(false, 64);
     }
