@@ -96,6 +96,38 @@ __device__ __forceinline__ float load_logit(const void* row, int32_t v, int is_b
 }
 
 // ---------------------------------------------------------------------------------------------
+// Shared-memory barriers (mbarrier).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Makes barrier initialisation visible to the other threads and to the copy engine.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
 // Warp / block reductions (blockDim.x == 32 * kWarpsPerBlock, all threads participate).
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float warp_max(float v) {
@@ -169,6 +201,42 @@ __device__ __forceinline__ void block_argmax(float& v, int& i, float* shv, int* 
     v = l < kWarps ? shv[l] : -INFINITY;
     i = l < kWarps ? shi[l] : 0x7fffffff;
     warp_argmax(v, i);
+}
+// Two independent (value, index) argmax reductions in one exchange; shv and shi hold 2 kWarps.
+template <int kWarps>
+__device__ __forceinline__ void block_argmax2(float& v0, int& i0, float& v1, int& i1, float* shv, int* shi) {
+    warp_argmax(v0, i0);
+    warp_argmax(v1, i1);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) {
+        shv[w] = v0;
+        shi[w] = i0;
+        shv[kWarps + w] = v1;
+        shi[kWarps + w] = i1;
+    }
+    __syncthreads();
+    v0 = l < kWarps ? shv[l] : -INFINITY;
+    i0 = l < kWarps ? shi[l] : 0x7fffffff;
+    v1 = l < kWarps ? shv[kWarps + l] : -INFINITY;
+    i1 = l < kWarps ? shi[kWarps + l] : 0x7fffffff;
+    warp_argmax(v0, i0);
+    warp_argmax(v1, i1);
+}
+// Two sums in one exchange; sh holds 2 kWarps.
+template <int kWarps>
+__device__ __forceinline__ void block_sum2(float& a, float& b, float* sh) {
+    a = warp_sum(a);
+    b = warp_sum(b);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) {
+        sh[w] = a;
+        sh[kWarps + w] = b;
+    }
+    __syncthreads();
+    a = warp_sum(l < kWarps ? sh[l] : 0.f);
+    b = warp_sum(l < kWarps ? sh[kWarps + l] : 0.f);
 }
 
 }  // namespace dg

@@ -6,10 +6,11 @@
 // epilogue, gives the log-sum-exp for the self-conditioning contraction and the canvas
 // cross-entropy L = -sum_i log p(x_0^i | ...).
 //
-// Phase 1 (all CTAs): each warp streams whole chunks of kChunk = 2048 consecutive ids of one row
-//   with 16-byte non-allocating loads (bf16: 8 loads of 16 B per lane, 512 B per warp-load),
-//   computes the chunk's raw maximum, S = sum exp(l' - m') and T = sum exp(l' - m')(l' - m') with
-//   l' = l * inv_tau and m' = max l', and writes one 16-byte record per chunk.
+// Phase 1 (all CTAs): each warp streams one group of 4 chunks (4 x kChunk = 2048 consecutive ids)
+//   of one row with 16-byte non-allocating loads (bf16: 8 loads of 16 B per lane, 512 B per
+//   warp-load); each 8-lane subgroup computes its chunk's raw maximum, S = sum exp(l' - m') and
+//   T = sum exp(l' - m')(l' - m') with l' = l * inv_tau and m' = max l', and writes one 16-byte
+//   record per chunk.
 // Phase 2 (the last CTA to finish a row, found by an atomic ticket -- nobody waits): merges the
 //   row's chunk records into lse, max-prob and entropy, finds the argmax, draws x0_hat by two-level
 //   Gumbel-max (level 1 over chunk records, level 2 by re-reading the winning chunk from L2), and
@@ -163,8 +164,8 @@ __device__ __noinline__ ChunkStats group_ragged(const void* row, bool bf16, int3
 }
 
 struct MergeShared {
-    float f[kPassWarps];
-    int i[kPassWarps];
+    float f[2 * kPassWarps];
+    int i[2 * kPassWarps];
     int flag;
 };
 
@@ -173,6 +174,10 @@ struct MergeShared {
 // Philox call serves its four chunk Gumbel variates), then the two chunks that must be re-read
 // (the one holding the argmax and the level-1 winner), fetched together.  Rows of more than
 // 4 * kPassThreads chunks re-read their further records from L2 in each pass.
+//
+// Three block-wide exchanges: (1) the argmax over the chunk maxima and the level-1 winner, which
+// fixes both chunks to re-read, so their loads are in flight during (2) the log-sum-exp merge of
+// (S, T); (3) the argmax inside the argmax chunk and the level-2 winner.
 static_assert(kChunk == 4 * kPassThreads, "one chunk is re-read as four ids per thread");
 
 template <bool kBf16, int kKind>
@@ -183,7 +188,9 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const float4* rec = p.rec + static_cast<size_t>(row) * nch;
     const float nbig = neg_big(kBf16);
 
-    // Cross-entropy: the target logit is fetched alongside the records.
+    // Scalars needed at the very end, loaded first so their latency overlaps the merge.
+    int32_t xt = 0;
+    if (kKind == kPassSampler && tid == 0) xt = p.x_t[row];
     float target_logit = 0.f;
     bool target_ok = false;
     int32_t b_seq = 0, i_seq = 0;
@@ -216,17 +223,61 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         }
     };
 
-    // Row maximum of the raw chunk maxima.
-    float mr = fmaxf(fmaxf(r[0].x, r[1].x), fmaxf(r[2].x, r[3].x));
+    // (1) The first chunk holding the row maximum of the raw chunk maxima, and the level-1 winner
+    // of the chunk scores lse_c + G_c (four chunks per Philox call).
+    const bool sampling = kKind == kPassSampler && p.mode != DG_X0_GREEDY;
+    float mv = -INFINITY, bs = -INFINITY;
+    int jm = 0x7fffffff, bj = 0x7fffffff;
+    auto scan_quad = [&](int32_t q, const float4 (&f)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (f[k].x > mv) {  // ascending ids, strict: the first maximum wins
+                mv = f[k].x;
+                jm = 4 * q + k;
+            }
+        if (sampling) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
+                p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int32_t j = 4 * q + k;
+                if (j < nch) {
+                    const float sc = (f[k].x * inv_tau + logf(f[k].y)) + gumbel_from_word(word_of(w, k));
+                    if (sc > bs) {
+                        bs = sc;
+                        bj = j;
+                    }
+                }
+            }
+        }
+    };
+    if (4 * tid < nch) scan_quad(tid, r);
     for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
         float4 f[4];
         far_quad(q, f);
-        mr = fmaxf(mr, fmaxf(fmaxf(f[0].x, f[1].x), fmaxf(f[2].x, f[3].x)));
+        scan_quad(q, f);
     }
-    const float m_raw = block_max<kPassWarps>(mr, sh.f);
+    block_argmax2<kPassWarps>(mv, jm, bs, bj, sh.f, sh.i);
+    const float m_raw = mv;
+    if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
+    if (!sampling || bj >= nch) bj = jm;  // greedy, or NaN scores only
     const float m_row = m_raw * inv_tau;
 
-    // Log-sum-exp merge of (S, T) relative to the row maximum.
+    // Both re-read chunks are known: ids lo + 4 tid .. lo + 4 tid + 3 of each, loaded now.
+    float av[4], gv[4];
+    const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
+    const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
+    if (kKind == kPassSampler) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int32_t va = alo + 4 * tid + k, vg = glo + 4 * tid + k;
+            av[k] = va < ahi ? fmaxf(load_logit(rowp, va, kBf16), nbig) : -INFINITY;
+            gv[k] = vg < ghi ? fmaxf(load_logit(rowp, vg, kBf16), nbig) : -INFINITY;
+        }
+    }
+
+    // (2) Log-sum-exp merge of (S, T) relative to the row maximum.
     float s = 0.f, t = 0.f;
     auto acc_st = [&](const float4& c) {
         if (c.x == -INFINITY) return;  // missing chunk
@@ -243,8 +294,8 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc_st(f[k]);
     }
-    const float S = block_sum<kPassWarps>(s, sh.f);
-    const float T = block_sum<kPassWarps>(t, sh.f);
+    block_sum2<kPassWarps>(s, t, sh.f);
+    const float S = s, T = t;
     const float ln_s = logf(S);
     const float lse = m_row + ln_s;
 
@@ -264,13 +315,14 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             p.row_ticket[row] = 0u;
             __threadfence();
             const unsigned prev = atomicAdd(&p.seq_ticket[b_seq], 1u);
-            sh.flag = prev == static_cast<unsigned>(p.C - 1);
+            const bool last = prev == static_cast<unsigned>(p.C - 1);
+            if (last) __threadfence();
+            sh.flag = last;
             sh.i[0] = b_seq;
         }
         __syncthreads();
         if (!sh.flag) return;
         const int32_t b = sh.i[0];
-        __threadfence();
         float acc = 0.f;
         for (int32_t q = tid; q < p.C; q += kPassThreads) acc += ld_cg_f(p.loss_rows + static_cast<int64_t>(b) * p.C + q);
         const float total = block_sum<kPassWarps>(acc, sh.f);
@@ -282,98 +334,39 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     }
 
     // ---- sampler epilogue
-    // argmax chunk: the first chunk whose raw maximum is the row maximum.
-    int jm = 0x7fffffff;
-#pragma unroll
-    for (int k = 3; k >= 0; --k)
-        if (r[k].x == m_raw) jm = 4 * tid + k;
-    for (int32_t q = tid + kPassThreads; 4 * q < nch && jm == 0x7fffffff; q += kPassThreads) {
-        float4 f[4];
-        far_quad(q, f);
-#pragma unroll
-        for (int k = 3; k >= 0; --k)
-            if (f[k].x == m_raw) jm = 4 * q + k;
-    }
-    jm = block_min_int<kPassWarps>(jm, sh.i);
-    if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
-
-    // Level 1: chunk scores lse_c + G_c, four chunks per Philox call.
-    int32_t bj = jm;
-    if (p.mode != DG_X0_GREEDY) {
-        float bs = -INFINITY;
-        int bjl = 0x7fffffff;
-        auto score_quad = [&](int32_t q, const float4 (&f)[4]) {
-            const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
-                p.key1);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int32_t j = 4 * q + k;
-                if (j < nch) {
-                    const float sc = (f[k].x * inv_tau + logf(f[k].y)) + gumbel_from_word(word_of(w, k));
-                    if (sc > bs) {
-                        bs = sc;
-                        bjl = j;
-                    }
-                }
-            }
-        };
-        if (4 * tid < nch) score_quad(tid, r);
-        for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
-            float4 f[4];
-            far_quad(q, f);
-            score_quad(q, f);
-        }
-        block_argmax<kPassWarps>(bs, bjl, sh.f, sh.i);
-        bj = bjl < nch ? bjl : jm;  // NaN scores only
-    }
-
-    // One round trip for both re-read chunks: ids lo + 4 tid .. lo + 4 tid + 3 of each.
-    const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
-    const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
-    float av[4], gv[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int32_t va = alo + 4 * tid + k, vg = glo + 4 * tid + k;
-        av[k] = va < ahi ? fmaxf(load_logit(rowp, va, kBf16), nbig) : -INFINITY;
-        gv[k] = vg < ghi ? fmaxf(load_logit(rowp, vg, kBf16), nbig) : -INFINITY;
-    }
+    // (3) The first id of the argmax chunk holding the row maximum, and the level-2 winner
+    // argmax of l'_v + G_v over the level-1 chunk (four ids per Philox call).
+    float amv = -INFINITY;
     int am = 0x7fffffff;
 #pragma unroll
-    for (int k = 3; k >= 0; --k)
-        if (alo + 4 * tid + k < ahi && av[k] == m_raw) am = alo + 4 * tid + k;
-    am = block_min_int<kPassWarps>(am, sh.i);
-    if (am >= p.V) am = jm * kChunk;
-
-    int32_t x0;
-    if (p.mode == DG_X0_GREEDY) {
-        x0 = am;
-    } else {
-        // Level 2: argmax of l'_v + G_v over the winning chunk, four ids per Philox call.
-        float bs2 = -INFINITY;
-        int bv = 0x7fffffff;
-        const int32_t vg0 = glo + 4 * tid;
-        if (vg0 < ghi) {
-            const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
-                p.key0, p.key1);
+    for (int k = 0; k < 4; ++k)
+        if (av[k] > amv) {
+            amv = av[k];
+            am = alo + 4 * tid + k;
+        }
+    float bs2 = -INFINITY;
+    int bv = 0x7fffffff;
+    const int32_t vg0 = glo + 4 * tid;
+    if (sampling && vg0 < ghi) {
+        const uint4 w = philox4x32_10(
+            make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel), p.key0,
+            p.key1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if (vg0 + k < ghi) {
-                    const float sc = gv[k] * inv_tau + gumbel_from_word(word_of(w, k));
-                    if (sc > bs2) {
-                        bs2 = sc;
-                        bv = vg0 + k;
-                    }
+        for (int k = 0; k < 4; ++k) {
+            if (vg0 + k < ghi) {
+                const float sc = gv[k] * inv_tau + gumbel_from_word(word_of(w, k));
+                if (sc > bs2) {
+                    bs2 = sc;
+                    bv = vg0 + k;
                 }
             }
         }
-        block_argmax<kPassWarps>(bs2, bv, sh.f, sh.i);
-        x0 = (bv >= glo && bv < ghi) ? bv : am;
     }
+    block_argmax2<kPassWarps>(amv, am, bs2, bv, sh.f, sh.i);
+    if (am < alo || am >= ahi) am = alo;
+    const int32_t x0 = sampling && bv >= glo && bv < ghi ? bv : am;
 
     if (tid == 0) {
-        const int32_t xt = p.x_t[row];
         unsigned long long t_stay, t_jump;
         if (x0 != xt) {
             t_stay = p.thr_stay_diff[canvas];
@@ -436,15 +429,17 @@ __global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_
     }
     // The barrier orders every warp's record stores before thread 0's fence, and the fence is
     // cumulative: one fence makes the whole CTA's records visible before its ticket increment.
+    // The last CTA of the row fences once more (acquire) before its threads read the records.
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(&p.row_ticket[row], 1u);
-        sh.flag = prev == static_cast<unsigned>(p.segs - 1);
+        const bool last = prev == static_cast<unsigned>(p.segs - 1);
+        if (last) __threadfence();
+        sh.flag = last;
     }
     __syncthreads();
     if (!sh.flag) return;
-    __threadfence();
     merge_row<kBf16, kKind>(p, row, canvas, inv_tau, rowp, sh);
 }
 

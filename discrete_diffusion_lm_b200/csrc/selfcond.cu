@@ -43,14 +43,14 @@ constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at the boost 
 
 struct alignas(64) KernelParams {
     CUtensorMap tm_logits;  // [R, V], box 128 rows x (64 bytes of ids)
-    CUtensorMap tm_E;       // [V, d], box 32 ids x 64 columns
+    CUtensorMap tm_E;       // [V, d], box kKBlock ids x 64 columns
     const float* lse;
     uint16_t* z;
     float* partial;
     int32_t R, C, V, d;
     int32_t n_tiles, splits, total_kb;
     long long wait_limit;  // cycles a wait may last before the CTA aborts
-    int32_t fault_block;   // test hook: the E copy of this 32-id block is never issued (-1: none)
+    int32_t fault_block;   // test hook: the E copy of this kKBlock-id block is never issued (-1: none)
     float inv_tau[DG_MAX_CANVASES];
 };
 
@@ -69,30 +69,6 @@ struct Cfg {
 };
 
 // ------------------------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 // Per-CTA wait control in shared memory: the abort flag every wait watches, and the wait limit.
 struct WaitCtl {
     int abort;
@@ -115,9 +91,6 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* 
             return false;
         }
     }
-}
-__device__ __forceinline__ void fence_barrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -268,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
     bid /= p.splits;
     const int nt = bid % p.n_tiles;
     const int mt = bid / p.n_tiles;
-    // Split s takes the 32-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
+    // Split s takes the kKBlock-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
     // few rows of E, so every E row is fetched by all its readers within a short window.
     const int kb0 = split;
     const int kstride = p.splits;
@@ -426,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
 // For 129 rows or more, a cluster of two CTAs shares each tile: tcgen05.mma.cta_group::2 with
 // M = 256 reads A (p) from both CTAs -- 128 rows each, from their own shared memory -- and B (E)
 // split by columns: each CTA stages only the half of every 256-column block that belongs to it,
-// so per 32-id stage a CTA loads 16 KB of E instead of 32 KB and the pipeline gets 8 stages.
+// so per stage of kKBlock ids a CTA loads half of the tile's E bytes and the rings get deeper.
 // The pair's accumulator is 128 TMEM lanes x kNT columns in each CTA (its own rows).
 // Signalling: both CTAs' E copies complete on the leader CTA's barrier (cta_group::2 TMA, no
 // multicast); the peer's softmax warps arrive remotely on the leader's p-ready barrier; the
@@ -546,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     bid /= p.splits;
     const int nt = bid % p.n_tiles;
     const int mp = bid / p.n_tiles;  // rows 256 mp .. 256 mp + 255; this CTA: 128 of them
-    // Split s takes the 32-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
+    // Split s takes the kKBlock-id blocks s, s + S, s + 2S, ...: at any moment all CTAs read the same
     // few rows of E, so every E row is fetched by all its readers within a short window.
     const int kb0 = split;
     const int kstride = p.splits;
