@@ -71,7 +71,10 @@ void dgo_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint3
 
 /* Counter domains (word 3 of the counter) -- a layout of our own, fixed
  * before any GPU code: the pages name no random-number generator. */
-enum { DOM_GUMBEL_TOKEN = 0, DOM_STEP = 1, DOM_NOISE = 2, DOM_CANVAS = 3, DOM_GUMBEL_CHUNK = 4 };
+enum {
+    DOM_GUMBEL_TOKEN = 0, DOM_STEP = 1, DOM_NOISE = 2, DOM_CANVAS = 3, DOM_GUMBEL_CHUNK = 4,
+    DOM_RENOISE = 5, DOM_SC_DROP = 6
+};
 
 static void philox_word4(uint64_t seed, uint32_t c0, uint32_t c1, uint32_t c2, uint32_t dom,
                          uint32_t out[4])
@@ -445,5 +448,188 @@ void dgo_canvas_ce(const float* logits, int64_t ld, const int32_t* x0, const int
             sum += loss;
         }
         loss_seq[b] = sum;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Temperature schedule [TR-Method, sampler paragraph: the temperature       */
+/* tau_t < 1 is annealed linearly over the denoising time scale from         */
+/* tau_max = 0.8 to tau_min = 0.4].  Reading: linear in t with tau(1) =      */
+/* tau_max (denoising starts at t = 1) and tau(0) = tau_min; t is clamped    */
+/* to [0, 1].                                                                */
+/* ------------------------------------------------------------------------ */
+double dgo_tau_linear(double t, double tau_max, double tau_min)
+{
+    if (t < 0.0) t = 0.0;
+    if (t > 1.0) t = 1.0;
+    return tau_min + (tau_max - tau_min) * t;
+}
+
+/* Fixed-point entropy used by the acceptance and stopping decisions:        */
+/* q = floor(H * 2^32) with H clamped to [0, 64] and NaN counted as 64.      */
+/* (Reading: the decisions compare sums of entropies against thresholds; in  */
+/* fixed point the sums are exact and independent of summation order.)      */
+static int64_t entropy_q(float h)
+{
+    double x = (double)h;
+    if (!(x >= 0.0)) x = isnan(x) ? 64.0 : 0.0;
+    if (x > 64.0) x = 64.0;
+    return (int64_t)floor(x * 4294967296.0);
+}
+
+/* Threshold ceil(x * 2^32) for a sum of fixed-point entropies ("sum < x").  */
+static int64_t entropy_threshold(double x)
+{
+    double y = ceil(x * 4294967296.0);
+    if (y > 9.0e18) return INT64_MAX;
+    if (y < 0.0) return 0;
+    return (int64_t)y;
+}
+
+typedef struct {
+    int64_t q;
+    int32_t i;
+} qpos;
+
+static int qpos_cmp(const void* a, const void* b)
+{
+    const qpos* x = (const qpos*)a;
+    const qpos* y = (const qpos*)b;
+    if (x->q != y->q) return x->q < y->q ? -1 : 1;
+    return x->i < y->i ? -1 : (x->i > y->i);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Entropy-bounded acceptance with uniform re-noising [TR-Method, sampler    */
+/* paragraph: tokens are accepted in ascending order of entropy so that a    */
+/* mutual-information bound stays strictly below an error tolerance; once    */
+/* the tolerance is reached, every other token is re-noised uniformly at     */
+/* random].  Reading (the pages give no formula for the bound): the bound of */
+/* an accepted set is the sum of its entropies, which bounds its total       */
+/* correlation from above.  Per canvas of C positions, positions are ordered */
+/* by ascending (q, position) and the k-th of that order is accepted iff     */
+/* q_1 + ... + q_k < ceil(eps * 2^32); a canvas whose lowest entropy is      */
+/* already >= eps accepts nothing.  Accepted positions take x0_hat, the      */
+/* others floor(w0 V / 2^32) from counter (0, row, step, DOM_RENOISE).       */
+/* H, x0_hat: [B*C]; outputs x_next [B*C], accepted [B*C] (0/1) and the      */
+/* number accepted per canvas n_acc [B].                                     */
+/* ------------------------------------------------------------------------ */
+void dgo_entropy_accept(const float* H, const int32_t* x0_hat, int32_t B, int32_t C, int32_t V,
+                        double eps, uint64_t seed, uint32_t step, int32_t* x_next,
+                        uint8_t* accepted, int32_t* n_acc)
+{
+    qpos* order = (qpos*)malloc(sizeof(qpos) * (size_t)C);
+    int64_t limit = entropy_threshold(eps);
+    uint32_t w[4];
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t r0 = (int64_t)b * C;
+        for (int32_t i = 0; i < C; ++i) {
+            order[i].q = entropy_q(H[r0 + i]);
+            order[i].i = i;
+            accepted[r0 + i] = 0;
+        }
+        qsort(order, (size_t)C, sizeof(qpos), qpos_cmp);
+        int64_t sum = 0;
+        int32_t n = 0;
+        for (int32_t k = 0; k < C; ++k) {
+            sum += order[k].q;
+            if (!(sum < limit)) break;
+            accepted[r0 + order[k].i] = 1;
+            ++n;
+        }
+        n_acc[b] = n;
+        for (int32_t i = 0; i < C; ++i) {
+            int64_t r = r0 + i;
+            if (accepted[r]) {
+                x_next[r] = x0_hat[r];
+            } else {
+                philox_word4(seed, 0u, (uint32_t)r, step, DOM_RENOISE, w);
+                x_next[r] = word_to_index(w[0], V);
+            }
+        }
+    }
+    free(order);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive stopping [TR-Method, sampler paragraph: early termination when   */
+/* the mean predicted entropy over the whole canvas falls below a threshold  */
+/* and the deterministic sequence predictions of two consecutive steps are   */
+/* identical].  Reading: the deterministic prediction is the argmax token of */
+/* each position; the mean uses the fixed-point entropies above, so the      */
+/* first condition is sum_i q_i < ceil(theta * C * 2^32).  Without a         */
+/* previous step (argmax_prev NULL) the second condition is false.           */
+/* Outputs stop [B] (0/1) and mean_H [B] = (sum_i q_i) 2^-32 / C.            */
+/* ------------------------------------------------------------------------ */
+void dgo_adaptive_stop(const float* H, const int32_t* am, const int32_t* am_prev, int32_t B,
+                       int32_t C, double theta, uint8_t* stop, double* mean_H)
+{
+    int64_t limit = entropy_threshold(theta * (double)C);
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t r0 = (int64_t)b * C;
+        int64_t sum = 0;
+        int same = am_prev != NULL;
+        for (int32_t i = 0; i < C; ++i) {
+            sum += entropy_q(H[r0 + i]);
+            if (am_prev && am[r0 + i] != am_prev[r0 + i]) same = 0;
+        }
+        mean_H[b] = (double)sum * (1.0 / 4294967296.0) / (double)C;
+        stop[b] = (uint8_t)(sum < limit && same);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Canvas cross-entropy backward [TR-Method, loss equation].  For row r with */
+/* target id y_r the derivative of loss_r = lse_r - l_r[y_r] is               */
+/*     d loss_r / d l_r[v] = softmax(l_r)_v - [v == y_r],                     */
+/* scaled by the upstream gradient g_seq[b] of the sequence's summed loss    */
+/* (rows b*C .. b*C+C-1).  lse is recomputed here in double.  A row whose    */
+/* target is out of range gets a zero gradient.                               */
+/* ------------------------------------------------------------------------ */
+void dgo_canvas_ce_backward(const float* logits, int64_t ld, const int32_t* x0,
+                            const int32_t* canvas_idx, int32_t n_seq, int32_t P, int32_t K,
+                            int32_t C, int32_t V, const double* g_seq, double* grad)
+{
+    int64_t L = (int64_t)P + (int64_t)K * C;
+    for (int32_t b = 0; b < n_seq; ++b) {
+        int32_t k = canvas_idx[b];
+        for (int32_t i = 0; i < C; ++i) {
+            int64_t r = (int64_t)b * C + i;
+            const float* l = logits + r * ld;
+            double* g = grad + r * (int64_t)V;
+            int32_t y = (k >= 0 && k < K) ? x0[(int64_t)b * L + P + (int64_t)k * C + i] : -1;
+            if (y < 0 || y >= V) {
+                for (int32_t v = 0; v < V; ++v) g[v] = 0.0;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int32_t v = 0; v < V; ++v)
+                if ((double)l[v] > m) m = (double)l[v];
+            double S = 0.0;
+            for (int32_t v = 0; v < V; ++v) S += exp((double)l[v] - m);
+            double lse = m + log(S);
+            for (int32_t v = 0; v < V; ++v)
+                g[v] = g_seq[b] * (exp((double)l[v] - lse) - (v == y ? 1.0 : 0.0));
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Self-conditioning drop for training [TR-Data: for 50% of the batch the    */
+/* decoder uses the self-conditioning state of a previous forward pass, for  */
+/* the other 50% that state is zero].  Reading: an independent fair coin per */
+/* sequence, keep iff w0 < 2^31 from counter (0, b, step, DOM_SC_DROP); the  */
+/* C rows of a dropped sequence are set to zero.  z: [n_seq*C, d] in place;   */
+/* keep [n_seq] (0/1).                                                       */
+/* ------------------------------------------------------------------------ */
+void dgo_selfcond_drop(double* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed,
+                       uint32_t step, uint8_t* keep)
+{
+    uint32_t w[4];
+    for (int32_t b = 0; b < n_seq; ++b) {
+        philox_word4(seed, 0u, (uint32_t)b, step, DOM_SC_DROP, w);
+        keep[b] = (uint8_t)(w[0] < 0x80000000u);
+        if (!keep[b])
+            for (int64_t j = (int64_t)b * C * d; j < ((int64_t)b + 1) * C * d; ++j) z[j] = 0.0;
     }
 }

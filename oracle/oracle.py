@@ -75,6 +75,12 @@ def _declare(L):
     L.dgo_selfcond_rows.argtypes = [_p, _i64, _i32, _p, _i32, _p, _p, _i32, _p]
     L.dgo_forward_noise.argtypes = [_p, _i32, _i32, _i32, _i32, _i32, _i32, _p, _u64, _p, _p]
     L.dgo_canvas_ce.argtypes = [_p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p]
+    L.dgo_tau_linear.argtypes = [_f64, _f64, _f64]
+    L.dgo_tau_linear.restype = _f64
+    L.dgo_entropy_accept.argtypes = [_p, _p, _i32, _i32, _i32, _f64, _u64, _u32, _p, _p, _p]
+    L.dgo_adaptive_stop.argtypes = [_p, _p, _p, _i32, _i32, _f64, _p, _p]
+    L.dgo_canvas_ce_backward.argtypes = [_p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p]
+    L.dgo_selfcond_drop.argtypes = [_p, _i32, _i32, _i32, _u64, _u32, _p]
 
 
 def _ptr(a: np.ndarray):
@@ -215,3 +221,51 @@ def canvas_ce(logits, x0, canvas_idx, n_seq: int, P: int, K: int, C: int, V: int
     lib().dgo_canvas_ce(_ptr(L), L.shape[1], _ptr(x), _ptr(k), n_seq, P, K, C, V, _ptr(loss),
                         _ptr(seq), _ptr(lse))
     return loss, seq, lse
+
+
+# --------------------------------------------------------------------------- sampler extensions
+def tau_linear(t: float, tau_max: float = 0.8, tau_min: float = 0.4) -> float:
+    """Linearly annealed temperature: tau(1) = tau_max, tau(0) = tau_min."""
+    return lib().dgo_tau_linear(float(t), float(tau_max), float(tau_min))
+
+
+def entropy_accept(H, x0_hat, B: int, C: int, V: int, eps: float, seed: int, step: int):
+    """Entropy-bounded acceptance per canvas; returns (x_next, accepted, n_accepted)."""
+    h = _f32(H)
+    x = _i32a(x0_hat)
+    out = np.zeros(B * C, dtype=np.int32)
+    acc = np.zeros(B * C, dtype=np.uint8)
+    n = np.zeros(B, dtype=np.int32)
+    lib().dgo_entropy_accept(_ptr(h), _ptr(x), B, C, V, float(eps), seed, step, _ptr(out), _ptr(acc), _ptr(n))
+    return out, acc, n
+
+
+def adaptive_stop(H, argmax, argmax_prev, B: int, C: int, theta: float):
+    """Adaptive-stopping flags per canvas; returns (stop, mean_entropy)."""
+    h = _f32(H)
+    a = _i32a(argmax)
+    ap = None if argmax_prev is None else _i32a(argmax_prev)
+    stop = np.zeros(B, dtype=np.uint8)
+    mean = np.zeros(B, dtype=np.float64)
+    lib().dgo_adaptive_stop(_ptr(h), _ptr(a), None if ap is None else _ptr(ap), B, C, float(theta), _ptr(stop),
+                            _ptr(mean))
+    return stop, mean
+
+
+def canvas_ce_backward(logits, x0, canvas_idx, n_seq: int, P: int, K: int, C: int, V: int, g_seq=None):
+    """d(sum_i loss_i of sequence b) * g_seq[b] / d logits, in double: [n_seq*C, V]."""
+    L = _f32(logits)
+    x = _i32a(x0)
+    k = _i32a(canvas_idx)
+    g = _f64a(np.ones(n_seq) if g_seq is None else g_seq)
+    out = np.zeros((n_seq * C, V), dtype=np.float64)
+    lib().dgo_canvas_ce_backward(_ptr(L), L.shape[1], _ptr(x), _ptr(k), n_seq, P, K, C, V, _ptr(g), _ptr(out))
+    return out
+
+
+def selfcond_drop(z, n_seq: int, C: int, d: int, seed: int, step: int):
+    """Zero the self-conditioning rows of dropped sequences; returns (z, keep)."""
+    zz = np.array(z, dtype=np.float64, copy=True, order="C")
+    keep = np.zeros(n_seq, dtype=np.uint8)
+    lib().dgo_selfcond_drop(_ptr(zz), n_seq, C, d, seed, step, _ptr(keep))
+    return zz, keep
