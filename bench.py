@@ -275,8 +275,9 @@ def run_ours(args, rank, world, local):
     roof["frac_of_slower_bound"] = round(max(t_tensor_us, t_hbm_us) / k2_mean, 4)
     k1_gbs = bytes_k1 / (k1_mean * 1e-6) / 1e9
 
-    # ---- training-side kernels on the training workload (forward noise + canvas CE)
+    # ---- training-side kernels on the training workload (forward noise + canvas CE + backward)
     train = bench_train(dg, W, dev, stream, hbm)
+    eb = bench_eb(dg, W, dev, stream, bufs, hbm)
 
     # ---- end to end through the public API with host buffers
     e2e = bench_e2e(dg, W, cfg, dev, E, args, world, barrier)
@@ -309,6 +310,7 @@ def run_ours(args, rank, world, local):
             "selfcond_frac_tensor_sustained": round(flops_k2 / (k2_mean * 1e-6) / 1e12 / tc, 4),
             "selfcond_frac_hbm": round(bytes_k2 / (k2_mean * 1e-6) / 1e9 / hbm, 4),
             "train": train,
+            "entropy_bounded": eb,
         },
         "e2e": e2e,
         "gpu_launches": int(round(launches_per_step * K)),
@@ -358,11 +360,87 @@ def bench_train(dg, W, dev, stream, hbm):
     noise_us = e[0].elapsed_time(e[1]) * 1e3 / reps
     ce_us = e[1].elapsed_time(e[2]) * 1e3 / reps
     ce_bytes = cfg.n_seq * cfg.C * cfg.V * 2
+    # backward of the canvas CE, in place over the same logits (their values no longer matter for
+    # timing), and the self-conditioning drop on a z of the training rows
+    z = torch.randn(cfg.n_seq * cfg.C, 2048, device=dev).to(torch.bfloat16)
+    gb, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        dg.dg_canvas_ce_backward(logits, lse, x0, kidx, cfg.P, cfg.K, cfg.C, stream=stream)
+        dg.dg_selfcond_drop(z, cfg.C, seed=0, step=0, stream=stream)
+    stream.synchronize()
+    with torch.cuda.graph(gb, stream=stream):
+        dg.dg_canvas_ce_backward(logits, lse, x0, kidx, cfg.P, cfg.K, cfg.C, stream=stream)
+    with torch.cuda.graph(gd, stream=stream):
+        dg.dg_selfcond_drop(z, cfg.C, seed=0, step=1, stream=stream)
+    e2 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gb.replay()
+            gd.replay()
+        e2[0].record(stream)
+        for _ in range(reps):
+            gb.replay()
+        e2[1].record(stream)
+        for _ in range(reps):
+            gd.replay()
+        e2[2].record(stream)
+    stream.synchronize()
+    bw_us = e2[0].elapsed_time(e2[1]) * 1e3 / reps
+    drop_us = e2[1].elapsed_time(e2[2]) * 1e3 / reps
+    bw_bytes = 2 * ce_bytes  # read and write every logit
     return {"workload": "train: 8 seq x (P=512 + K=4 x C=256), V=262144, bf16 CE logits [2048, 262144]",
             "forward_noise_us": round(noise_us, 2), "canvas_ce_us": round(ce_us, 2),
             "canvas_ce_GBps": round(ce_bytes / (ce_us * 1e-6) / 1e9, 1),
             "canvas_ce_frac_hbm": round(ce_bytes / (ce_us * 1e-6) / 1e9 / hbm, 4),
-            "note": "canvas CE logits (1.07 GB) exceed L2; repeated on one buffer"}
+            "ce_backward_us": round(bw_us, 2),
+            "ce_backward_GBps": round(bw_bytes / (bw_us * 1e-6) / 1e9, 1),
+            "ce_backward_frac_hbm": round(bw_bytes / (bw_us * 1e-6) / 1e9 / hbm, 4),
+            "selfcond_drop_us": round(drop_us, 2),
+            "note": "canvas CE logits (1.07 GB) exceed L2; repeated on one buffer (the backward in place)"}
+
+
+def bench_eb(dg, W, dev, stream, bufs, hbm):
+    """The entropy-bounded sampler step (logits pass + per-canvas acceptance and stopping) on the
+    full-vocab workload with the annealed temperature, and the per-canvas kernel alone."""
+    import torch
+    cfg = W.FULL
+    nbuf = len(bufs)
+    outs = [dg.dg_sampler_step_eb(bufs[0], cfg.C, eps=64.0, theta=0.5, inv_tau=dg.dg_tau_linear([0.5]), stream=stream)
+            for _ in range(2)]
+    ws = torch.zeros(dg.dg_sampler_step_workspace_size(cfg.R, cfg.V), dtype=torch.uint8, device=dev)
+    graphs = []
+    stream.synchronize()
+    for k in range(nbuf):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            dg.dg_sampler_step_eb(bufs[k], cfg.C, eps=64.0, theta=0.5, argmax_prev=outs[(k + 1) % 2]["argmax"],
+                                  inv_tau=dg.dg_tau_linear([1.0 - k / nbuf]), seed=0, step=k, out=outs[k % 2],
+                                  ws=ws, stream=stream)
+        graphs.append(g)
+    gdec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gdec, stream=stream):
+        dg.dg_entropy_accept(outs[0]["entropy"], outs[0]["x0_hat"], cfg.C, cfg.V, 64.0, stream=stream)
+    reps = 24
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        for k in range(4):
+            graphs[k % nbuf].replay()
+            gdec.replay()
+        e[0].record(stream)
+        for k in range(reps):
+            graphs[k % nbuf].replay()
+        e[1].record(stream)
+        for k in range(reps):
+            gdec.replay()
+        e[2].record(stream)
+    stream.synchronize()
+    step_us = e[0].elapsed_time(e[1]) * 1e3 / reps
+    dec_us = e[1].elapsed_time(e[2]) * 1e3 / reps
+    lbytes = cfg.R * cfg.V * 2
+    return {"workload": "entropy-bounded step on the full-vocab workload (C=256, V=262144), eps=64, theta=0.5, "
+                        "tau annealed 0.8->0.4", "eb_step_us": round(step_us, 2),
+            "eb_step_frac_hbm": round(lbytes / (step_us * 1e-6) / 1e9 / hbm, 4),
+            "canvas_decide_us": round(dec_us, 2)}
 
 
 def bench_e2e(dg, W, cfg, dev, E, args, world, barrier):

@@ -67,6 +67,13 @@ def lib() -> ctypes.CDLL:
         L.dg_canvas_ce_workspace_size.argtypes = [_i32, _i32, _i32]
         L.dg_canvas_ce_workspace_size.restype = _sz
         L.dg_canvas_ce.argtypes = [_p, _int, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _sz, _p]
+        L.dg_tau_linear.argtypes = [_p, _i32, ctypes.c_double, ctypes.c_double, _p]
+        L.dg_entropy_accept.argtypes = [_p, _p, _i32, _i32, _i32, ctypes.c_double, _u64, _u32, _p, _p, _p, _p]
+        L.dg_adaptive_stop.argtypes = [_p, _p, _p, _i32, _i32, ctypes.c_double, _p, _p, _p]
+        L.dg_sampler_step_eb.argtypes = [_p, _int, _i64, _i32, _i32, _i32, _p, _u64, _u32, _int, ctypes.c_double,
+                                         ctypes.c_double, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]
+        L.dg_canvas_ce_backward.argtypes = [_p, _i64, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p]
+        L.dg_selfcond_drop.argtypes = [_p, _i32, _i32, _i32, _u64, _u32, _p, _p]
         _lib = L
     return _lib
 
@@ -309,3 +316,114 @@ def dg_canvas_ce(logits: torch.Tensor, x0: torch.Tensor, canvas_idx: torch.Tenso
                             ws.numel() * ws.element_size(), _stream(stream))
     _check("dg_canvas_ce", rc)
     return loss_rows, loss_seq, lse_rows
+
+
+# ------------------------------------------------------------------------------ sampler extensions
+def dg_tau_linear(t, tau_max: float = 0.8, tau_min: float = 0.4) -> list:
+    """Per-canvas inverse temperatures of the linear schedule tau(1) = tau_max, tau(0) = tau_min."""
+    tt = _expand(t, 1) if isinstance(t, (int, float)) else list(t)
+    n = len(tt)
+    out = (ctypes.c_float * n)()
+    rc = lib().dg_tau_linear(_host_doubles(tt, n), n, float(tau_max), float(tau_min), out)
+    _check("dg_tau_linear", rc)
+    return [float(v) for v in out]
+
+
+def dg_entropy_accept(entropy: torch.Tensor, x0_hat: torch.Tensor, C: int, V: int, eps: float, *, seed: int = 0,
+                      step: int = 0, out: Optional[dict] = None, stream=None) -> dict:
+    """Entropy-bounded acceptance per canvas; returns {x_next, accepted, n_accepted}."""
+    R = entropy.numel()
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = entropy.device
+    if out is None:
+        out = {"x_next": torch.empty(R, dtype=torch.int32, device=dev),
+               "accepted": torch.empty(R, dtype=torch.uint8, device=dev),
+               "n_accepted": torch.empty(B, dtype=torch.int32, device=dev)}
+    rc = lib().dg_entropy_accept(_ptr(entropy), _ptr(x0_hat), B, C, V, float(eps), ctypes.c_uint64(seed),
+                                 ctypes.c_uint32(step), _ptr(out["x_next"]), _ptr(out.get("accepted")),
+                                 _ptr(out.get("n_accepted")), _stream(stream))
+    _check("dg_entropy_accept", rc)
+    return out
+
+
+def dg_adaptive_stop(entropy: torch.Tensor, argmax: torch.Tensor, argmax_prev: Optional[torch.Tensor], C: int,
+                     theta: float, *, stream=None):
+    """Adaptive-stopping flags per canvas; returns (stop uint8 [B], mean_entropy float [B])."""
+    R = entropy.numel()
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    stop = torch.empty(B, dtype=torch.uint8, device=entropy.device)
+    mean = torch.empty(B, dtype=torch.float32, device=entropy.device)
+    rc = lib().dg_adaptive_stop(_ptr(entropy), _ptr(argmax), _ptr(argmax_prev), B, C, float(theta), _ptr(stop),
+                                _ptr(mean), _stream(stream))
+    _check("dg_adaptive_stop", rc)
+    return stop, mean
+
+
+def dg_sampler_step_eb(logits: torch.Tensor, C: int, *, eps: float, theta: float = 0.0,
+                       argmax_prev: Optional[torch.Tensor] = None, V: Optional[int] = None, inv_tau=None,
+                       seed: int = 0, step: int = 0, mode: str = "sample", out: Optional[dict] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Entropy-bounded sampler step: statistics and x0_hat draw, then per-canvas acceptance with
+    uniform re-noising and the adaptive-stopping flag.  Returns the dict of outputs (x_next,
+    x0_hat, argmax, max_prob, lse, entropy, accepted, stop, mean_entropy)."""
+    ld = _row_major_2d(logits, "logits")
+    R = logits.shape[0]
+    V = logits.shape[1] if V is None else V
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = logits.device
+    if out is None:
+        out = {k: torch.empty(R, dtype=dt, device=dev) for k, dt in
+               (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32),
+                ("max_prob", torch.float32), ("lse", torch.float32), ("entropy", torch.float32),
+                ("accepted", torch.uint8))}
+        out["stop"] = torch.empty(B, dtype=torch.uint8, device=dev)
+        out["mean_entropy"] = torch.empty(B, dtype=torch.float32, device=dev)
+    nbytes = dg_sampler_step_workspace_size(R, V)
+    if ws is None:
+        ws = workspace("sampler_step", nbytes, dev, (R, V), stream)
+    rc = lib().dg_sampler_step_eb(
+        _ptr(logits), _dtype_code(logits), ld, B, C, V, _host_floats(None if inv_tau is None else _expand(inv_tau, B), B),
+        ctypes.c_uint64(seed), ctypes.c_uint32(step), DG_X0[mode], float(eps), float(theta), _ptr(argmax_prev),
+        _ptr(out["x_next"]), _ptr(out["x0_hat"]), _ptr(out.get("argmax")), _ptr(out.get("max_prob")),
+        _ptr(out.get("lse")), _ptr(out["entropy"]), _ptr(out.get("accepted")), _ptr(out.get("stop")),
+        _ptr(out.get("mean_entropy")), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("dg_sampler_step_eb", rc)
+    return out
+
+
+def dg_canvas_ce_backward(logits: torch.Tensor, lse_rows: torch.Tensor, x0: torch.Tensor, canvas_idx: torch.Tensor,
+                          P: int, K: int, C: int, *, V: Optional[int] = None, g_seq: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Overwrite bf16 logits with d(sum of each sequence's canvas CE) / d logits (times g_seq)."""
+    ld = _row_major_2d(logits, "logits")
+    if logits.dtype != torch.bfloat16:
+        raise TypeError("the in-place CE backward works on bf16 logits")
+    V = logits.shape[1] if V is None else V
+    n_seq = x0.shape[0]
+    rc = lib().dg_canvas_ce_backward(_ptr(logits), ld, _ptr(lse_rows), _ptr(x0), _ptr(canvas_idx), n_seq, P, K, C, V,
+                                     _ptr(g_seq), _stream(stream))
+    _check("dg_canvas_ce_backward", rc)
+    return logits
+
+
+def dg_selfcond_drop(z: torch.Tensor, C: int, *, seed: int = 0, step: int = 0,
+                     keep: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Zero, in place, the bf16 self-conditioning rows of sequences whose fair coin drops them;
+    returns keep (uint8 [n_seq])."""
+    if z.dtype != torch.bfloat16 or not z.is_contiguous():
+        raise TypeError("z must be a contiguous bf16 tensor [n_seq*C, d]")
+    R, d = z.shape
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    n_seq = R // C
+    keep = torch.empty(n_seq, dtype=torch.uint8, device=z.device) if keep is None else keep
+    rc = lib().dg_selfcond_drop(_ptr(z), n_seq, C, d, ctypes.c_uint64(seed), ctypes.c_uint32(step), _ptr(keep),
+                                _stream(stream))
+    _check("dg_selfcond_drop", rc)
+    return keep

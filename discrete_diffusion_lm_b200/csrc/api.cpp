@@ -97,6 +97,15 @@ void step_thresholds(int schedule, double t, double dt, int32_t V, unsigned long
     *stay_same = prob_threshold(1.0 - uniform);
 }
 
+// Threshold for sums of fixed-point entropies q = floor(H 2^32): (sum q < T) <=> (sum q < x 2^32),
+// T = ceil(x 2^32) (x 2^32 is exact in double), clamped to [0, 2^63).
+long long entropy_threshold(double x) {
+    if (!(x > 0.0)) return 0;
+    const double y = std::ceil(x * 4294967296.0);
+    if (y >= 9.0e18) return 0x7fffffffffffffffLL;
+    return static_cast<long long>(y);
+}
+
 int32_t n_chunks_of(int32_t V) { return (V + kChunk - 1) / kChunk; }
 
 // Groups of 4 chunks (2048 ids) per CTA of the logits pass: one per warp.
@@ -460,6 +469,195 @@ int dg_test_selfcond_stall(const void* logits, int logits_dtype, int64_t ld, int
     }
     return selfcond_impl(logits, logits_dtype, ld, B, C, V, inv_tau, lse, E, embed_dtype, d, z, workspace,
                          workspace_bytes, stream, stalled_block, static_cast<long long>(limit_cycles));
+}
+
+
+int dg_tau_linear(const double* t, int32_t B, double tau_max, double tau_min, float* inv_tau) {
+    g_last_error.clear();
+    if (!t || !inv_tau) return fail(DG_ERR_INVALID_ARG, "t and inv_tau (host arrays) are required");
+    if (B < 1) return fail(DG_ERR_INVALID_ARG, "B = %d must be >= 1", B);
+    if (!(tau_min > 0.0) || !(tau_max > 0.0) || !std::isfinite(tau_min) || !std::isfinite(tau_max))
+        return fail(DG_ERR_INVALID_ARG, "tau_max = %g and tau_min = %g must be finite and > 0", tau_max, tau_min);
+    for (int32_t b = 0; b < B; ++b) {
+        double x = t[b];
+        if (std::isnan(x)) return fail(DG_ERR_INVALID_ARG, "t[%d] is NaN", b);
+        x = x < 0.0 ? 0.0 : (x > 1.0 ? 1.0 : x);
+        inv_tau[b] = static_cast<float>(1.0 / (tau_min + (tau_max - tau_min) * x));
+    }
+    return DG_OK;
+}
+
+int dg_entropy_accept(const float* entropy, const int32_t* x0_hat, int32_t B, int32_t C, int32_t V, double eps,
+                      uint64_t seed, uint32_t step, int32_t* x_next, uint8_t* accepted, int32_t* n_accepted,
+                      dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if (!entropy || !x0_hat || !x_next) return fail(DG_ERR_INVALID_ARG, "entropy, x0_hat and x_next are required");
+    if ((rc = check_canvases(B, C)) != DG_OK) return rc;
+    if (C > DG_MAX_CANVAS_ROWS) return fail(DG_ERR_UNSUPPORTED, "C = %d exceeds %d", C, DG_MAX_CANVAS_ROWS);
+    if (V < 1) return fail(DG_ERR_INVALID_ARG, "V = %d must be >= 1", V);
+    if (std::isnan(eps)) return fail(DG_ERR_INVALID_ARG, "eps is NaN");
+    if ((rc = check_device()) != DG_OK) return rc;
+    DecideParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.entropy = entropy;
+    p.x0_hat = x0_hat;
+    p.C = C;
+    p.V = V;
+    p.accept_limit = entropy_threshold(eps);
+    p.key0 = static_cast<uint32_t>(seed);
+    p.key1 = static_cast<uint32_t>(seed >> 32);
+    p.step = step;
+    p.x_next = x_next;
+    p.accepted = accepted;
+    p.n_accepted = n_accepted;
+    const cudaError_t e = launch_canvas_decide(p, B, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "acceptance launch");
+    return DG_OK;
+}
+
+int dg_adaptive_stop(const float* entropy, const int32_t* argmax, const int32_t* argmax_prev, int32_t B, int32_t C,
+                     double theta, uint8_t* stop, float* mean_entropy, dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if (!entropy || !argmax) return fail(DG_ERR_INVALID_ARG, "entropy and argmax are required");
+    if (!stop && !mean_entropy) return fail(DG_ERR_INVALID_ARG, "no output requested");
+    if ((rc = check_canvases(B, C)) != DG_OK) return rc;
+    if (C > DG_MAX_CANVAS_ROWS) return fail(DG_ERR_UNSUPPORTED, "C = %d exceeds %d", C, DG_MAX_CANVAS_ROWS);
+    if (std::isnan(theta)) return fail(DG_ERR_INVALID_ARG, "theta is NaN");
+    if ((rc = check_device()) != DG_OK) return rc;
+    DecideParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.entropy = entropy;
+    p.argmax = argmax;
+    p.argmax_prev = argmax_prev;
+    p.C = C;
+    p.stop_limit = entropy_threshold(theta * static_cast<double>(C));
+    p.stop = stop;
+    p.mean_entropy = mean_entropy;
+    const cudaError_t e = launch_canvas_decide(p, B, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stopping launch");
+    return DG_OK;
+}
+
+int dg_sampler_step_eb(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
+                       const float* inv_tau, uint64_t seed, uint32_t step, int x0_mode, double eps, double theta,
+                       const int32_t* argmax_prev, int32_t* x_next, int32_t* x0_hat, int32_t* argmax,
+                       float* max_prob, float* lse, float* entropy, uint8_t* accepted, uint8_t* stop,
+                       float* mean_entropy, void* workspace, size_t workspace_bytes, dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if ((rc = check_logits(logits, logits_dtype, ld, V)) != DG_OK) return rc;
+    if ((rc = check_canvases(B, C)) != DG_OK) return rc;
+    if (C > DG_MAX_CANVAS_ROWS) return fail(DG_ERR_UNSUPPORTED, "C = %d exceeds %d", C, DG_MAX_CANVAS_ROWS);
+    if (!x_next || !x0_hat || !entropy) return fail(DG_ERR_INVALID_ARG, "x_next, x0_hat and entropy are required");
+    if ((stop || mean_entropy) && !argmax) return fail(DG_ERR_INVALID_ARG, "stopping needs the argmax output");
+    if (x0_mode != DG_X0_SAMPLE && x0_mode != DG_X0_GREEDY)
+        return fail(DG_ERR_INVALID_ARG, "x0_mode %d is not SAMPLE or GREEDY", x0_mode);
+    if (std::isnan(eps) || std::isnan(theta)) return fail(DG_ERR_INVALID_ARG, "eps and theta may not be NaN");
+    const int32_t R = B * C;
+    const size_t need = pass_ws_bytes(R, V, 0);
+    if (!workspace || workspace_bytes < need)
+        return fail(DG_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(DG_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+    static thread_local PassParams p;
+    std::memset(&p, 0, sizeof(p));
+    if ((rc = check_inv_tau(inv_tau, B, p.inv_tau)) != DG_OK) return rc;
+    if ((rc = check_device()) != DG_OK) return rc;
+    const PassWs w = carve_pass_ws(workspace, R, 0);
+    p.logits = logits;
+    p.ld = ld;
+    p.R = R;
+    p.C = C;
+    p.V = V;
+    p.n_chunks = n_chunks_of(V);
+    p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
+    p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
+    p.rec = w.rec;
+    p.row_ticket = w.row_ticket;
+    p.key0 = static_cast<uint32_t>(seed);
+    p.key1 = static_cast<uint32_t>(seed >> 32);
+    p.step = step;
+    p.mode = x0_mode;
+    p.x0_hat = x0_hat;  // x_next stays null: the per-canvas rule below decides it
+    p.argmax = argmax;
+    p.max_prob = max_prob;
+    p.lse = lse;
+    p.entropy = entropy;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_logits_pass(p, kPassSampler, logits_dtype == DG_BF16, st);
+    if (e != cudaSuccess) return cuda_fail(e, "logits pass launch");
+    DecideParams d;
+    std::memset(&d, 0, sizeof(d));
+    d.entropy = entropy;
+    d.x0_hat = x0_hat;
+    d.argmax = argmax;
+    d.argmax_prev = argmax_prev;
+    d.C = C;
+    d.V = V;
+    d.accept_limit = entropy_threshold(eps);
+    d.stop_limit = entropy_threshold(theta * static_cast<double>(C));
+    d.key0 = p.key0;
+    d.key1 = p.key1;
+    d.step = step;
+    d.x_next = x_next;
+    d.accepted = accepted;
+    d.stop = stop;
+    d.mean_entropy = mean_entropy;
+    e = launch_canvas_decide(d, B, st);
+    if (e != cudaSuccess) return cuda_fail(e, "per-canvas decision launch");
+    return DG_OK;
+}
+
+int dg_canvas_ce_backward(void* logits, int64_t ld, const float* lse_rows, const int32_t* x0,
+                          const int32_t* canvas_idx, int32_t n_seq, int32_t P, int32_t K, int32_t C, int32_t V,
+                          const float* g_seq, dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if ((rc = check_logits(logits, DG_BF16, ld, V)) != DG_OK) return rc;
+    if (!lse_rows || !x0 || !canvas_idx) return fail(DG_ERR_INVALID_ARG, "lse_rows, x0 and canvas_idx are required");
+    if (n_seq < 1 || n_seq > DG_MAX_CANVASES)
+        return fail(DG_ERR_INVALID_ARG, "n_seq = %d must be in [1, %d]", n_seq, DG_MAX_CANVASES);
+    if (P < 0 || K < 1 || C < 1) return fail(DG_ERR_INVALID_ARG, "need P >= 0, K >= 1, C >= 1");
+    if (V % 8 != 0) return fail(DG_ERR_ALIGNMENT, "V = %d must be a multiple of 8 (16-byte bf16 vectors)", V);
+    const long long L = static_cast<long long>(P) + static_cast<long long>(K) * C;
+    if (L > 0x7fffffffLL || static_cast<long long>(n_seq) * C > 0x7fffffffLL)
+        return fail(DG_ERR_INVALID_ARG, "sizes overflow int32");
+    if ((rc = check_device()) != DG_OK) return rc;
+    CeBackwardParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.logits = logits;
+    p.ld = ld;
+    p.lse = lse_rows;
+    p.x0 = x0;
+    p.canvas_idx = canvas_idx;
+    p.g_seq = g_seq;
+    p.R = n_seq * C;
+    p.C = C;
+    p.V = V;
+    p.P = P;
+    p.K = K;
+    p.seq_len = L;
+    const cudaError_t e = launch_ce_backward(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "CE backward launch");
+    return DG_OK;
+}
+
+int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed, uint32_t step, uint8_t* keep,
+                     dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if (!z) return fail(DG_ERR_INVALID_ARG, "z is NULL");
+    if (n_seq < 1 || C < 1 || d < 1) return fail(DG_ERR_INVALID_ARG, "need n_seq, C, d >= 1");
+    if (!aligned16(z)) return fail(DG_ERR_ALIGNMENT, "z is not 16-byte aligned");
+    const long long per_seq = static_cast<long long>(C) * d;
+    if (per_seq % 8 != 0) return fail(DG_ERR_ALIGNMENT, "C * d = %lld must be a multiple of 8", per_seq);
+    if ((rc = check_device()) != DG_OK) return rc;
+    const cudaError_t e = launch_selfcond_drop(static_cast<uint16_t*>(z), n_seq, per_seq, static_cast<uint32_t>(seed),
+                                               static_cast<uint32_t>(seed >> 32), step, keep,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-conditioning drop launch");
+    return DG_OK;
 }
 
 }  // extern "C"

@@ -1,0 +1,237 @@
+// Per-canvas sampler decisions and training-side elementwise passes.
+//
+// DiffusionGemma Technical Report (hyper.ai summary), section "Method", sampler paragraph:
+//   tokens are accepted in ascending order of entropy while an error bound stays strictly below
+//   a tolerance, the rest are re-noised uniformly at random; the sampler stops once the canvas-
+//   mean entropy is below a threshold and two consecutive deterministic predictions agree.
+// Same page, loss equation L = -sum_i log p(x0^i | x_t, z_t, H): its gradient with respect to
+//   the logits, softmax - one-hot, written over the logits in place.
+// Same page, section "Dataset": the self-conditioning state is used for half of the batch and
+//   zero for the other half.
+//
+// canvas_decide_kernel: one CTA of kDecideThreads threads per canvas (C <= DG_MAX_CANVAS_ROWS).
+//   Entropies become fixed-point integers q = floor(clamp(H, 0, 64) 2^32) (NaN -> 64), so sums
+//   and comparisons are exact and order-free.  Acceptance: ranks by (q, position) are computed by
+//   counting in shared memory, the rank-ordered q are prefix-summed (a block scan) and the
+//   accepted set is the ranks whose prefix is below the tolerance.  Stopping: the sum of q
+//   against the threshold, and an all-equal test of the argmax canvas against the previous one.
+// ce_backward_kernel: rows along grid y, 16-byte bf16 vectors of a row along grid x, in place.
+// selfcond_drop_kernel: one CTA per sequence; a fair Philox coin decides, dropped rows are zeroed.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dg {
+
+namespace {
+
+constexpr int kDecideThreads = 256;
+constexpr int kPerThread = (DG_MAX_CANVAS_ROWS + kDecideThreads - 1) / kDecideThreads;
+
+__device__ __forceinline__ long long entropy_q(float h) {
+    float x = h;
+    if (!(x >= 0.f)) x = isnan(x) ? 64.f : 0.f;
+    x = fminf(x, 64.f);
+    return __float2ll_rd(x * 4294967296.f);  // exact: a power-of-two scale of a float
+}
+
+// Inclusive block-wide prefix sum of one 64-bit value per thread.
+__device__ __forceinline__ long long block_inclusive_scan(long long v, long long* sh_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) sh_warp[warp] = v;
+    __syncthreads();
+    long long base = 0;
+    for (int w = 0; w < warp; ++w) base += sh_warp[w];
+    __syncthreads();
+    return v + base;
+}
+
+__global__ void __launch_bounds__(kDecideThreads) canvas_decide_kernel(const __grid_constant__ DecideParams p) {
+    __shared__ long long q[DG_MAX_CANVAS_ROWS];
+    __shared__ long long sorted[DG_MAX_CANVAS_ROWS];
+    __shared__ long long sh_warp[kDecideThreads / 32];
+    __shared__ int sh_count[kDecideThreads / 32];
+    __shared__ int sh_same;
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int C = p.C;
+    const int64_t r0 = static_cast<int64_t>(b) * C;
+    if (tid == 0) sh_same = 1;
+    for (int i = tid; i < C; i += kDecideThreads) q[i] = entropy_q(p.entropy[r0 + i]);
+    __syncthreads();
+
+    // ---- adaptive stopping: sum of q and the argmax comparison
+    if (p.stop || p.mean_entropy) {
+        long long s = 0;
+        int diff = 0;
+        for (int i = tid; i < C; i += kDecideThreads) {
+            s += q[i];
+            if (p.argmax_prev && p.argmax[r0 + i] != p.argmax_prev[r0 + i]) diff = 1;
+        }
+        if (__any_sync(0xffffffffu, diff) && (tid & 31) == 0) sh_same = 0;
+        const long long total = block_inclusive_scan(s, sh_warp);  // the last thread holds the sum
+        if (tid == kDecideThreads - 1) {
+            const bool same = p.argmax_prev != nullptr && sh_same != 0;
+            if (p.stop) p.stop[b] = static_cast<uint8_t>(total < p.stop_limit && same);
+            if (p.mean_entropy)
+                p.mean_entropy[b] = static_cast<float>(static_cast<double>(total) * (1.0 / 4294967296.0) /
+                                                       static_cast<double>(C));
+        }
+    }
+    if (!p.x_next) return;
+
+    // ---- entropy-bounded acceptance
+    int rank[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int i = tid + u * kDecideThreads;
+        rank[u] = 0;
+        if (i < C) {
+            const long long qi = q[i];
+            int r = 0;
+            for (int j = 0; j < C; ++j) {
+                const long long qj = q[j];
+                r += (qj < qi) | ((qj == qi) & (j < i));
+            }
+            rank[u] = r;
+            sorted[r] = qi;
+        }
+    }
+    __syncthreads();
+    // thread t scans ranks kPerThread t .. kPerThread t + kPerThread - 1
+    long long local[kPerThread];
+    long long run = 0;
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int k = tid * kPerThread + u;
+        run += k < C ? sorted[k] : 0;
+        local[u] = run;
+    }
+    const long long incl = block_inclusive_scan(run, sh_warp);
+    const long long base = incl - run;
+    int cnt = 0;
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int k = tid * kPerThread + u;
+        cnt += (k < C) & (base + local[u] < p.accept_limit);
+    }
+    // the accepted ranks are a prefix (q >= 0): their number is the count of passing prefixes
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if ((tid & 31) == 0) sh_count[tid >> 5] = cnt;
+    __syncthreads();
+    int n_acc = 0;
+#pragma unroll
+    for (int w = 0; w < kDecideThreads / 32; ++w) n_acc += sh_count[w];
+    if (tid == 0 && p.n_accepted) p.n_accepted[b] = n_acc;
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int i = tid + u * kDecideThreads;
+        if (i < C) {
+            const int64_t r = r0 + i;
+            const bool acc = rank[u] < n_acc;
+            int32_t x;
+            if (acc) {
+                x = p.x0_hat[r];
+            } else {
+                const uint4 w = philox4x32_10(
+                    make_uint4(0u, static_cast<uint32_t>(r), p.step, kDomRenoise), p.key0, p.key1);
+                x = word_to_index(w.x, p.V);
+            }
+            p.x_next[r] = x;
+            if (p.accepted) p.accepted[r] = static_cast<uint8_t>(acc);
+        }
+    }
+}
+
+// grad = g_seq[b] (exp(l - lse) - [v == y]) over bf16 rows, in place.  Grid: x covers a row's
+// 16-byte vectors (8 ids each), kCeVec per thread, consecutive threads on consecutive vectors;
+// y strides over rows.
+constexpr int kCeVec = 4;
+__global__ void __launch_bounds__(256) ce_backward_kernel(const __grid_constant__ CeBackwardParams p) {
+    const int32_t vec_per_row = p.V / 8;
+    for (int32_t r = blockIdx.y; r < p.R; r += gridDim.y) {
+        const int32_t b = r / p.C, i = r - b * p.C;
+        const int32_t k = p.canvas_idx[b];
+        int32_t y = -1;
+        if (k >= 0 && k < p.K) y = p.x0[static_cast<int64_t>(b) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i];
+        uint4* row = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.logits) + static_cast<int64_t>(r) * p.ld);
+        const int32_t v_base = blockIdx.x * (kCeVec * 256) + threadIdx.x;
+        if (y < 0 || y >= p.V) {
+#pragma unroll
+            for (int u = 0; u < kCeVec; ++u) {
+                const int32_t vi = v_base + u * 256;
+                if (vi < vec_per_row) row[vi] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            continue;
+        }
+        const float g = p.g_seq ? p.g_seq[b] : 1.0f;
+        const float nb = -p.lse[r] * kLog2e;
+        uint4 in[kCeVec];
+#pragma unroll
+        for (int u = 0; u < kCeVec; ++u) {
+            const int32_t vi = v_base + u * 256;
+            in[u] = vi < vec_per_row ? row[vi] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kCeVec; ++u) {
+            const int32_t vi = v_base + u * 256;
+            if (vi >= vec_per_row) continue;
+            const uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int32_t v = vi * 8 + 2 * j;
+                float lo = g * ex2_approx(fmaf(bf16_lo(w[j]), kLog2e, nb));
+                float hi = g * ex2_approx(fmaf(bf16_hi(w[j]), kLog2e, nb));
+                if (v == y) lo -= g;
+                if (v + 1 == y) hi -= g;
+                o[j] = pack_bf16x2(lo, hi);
+            }
+            row[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) selfcond_drop_kernel(uint16_t* z, int64_t seq_elems, uint32_t key0,
+                                                            uint32_t key1, uint32_t step, uint8_t* keep) {
+    const int b = blockIdx.x;
+    const uint4 w = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(b), step, kDomScDrop), key0, key1);
+    const bool kept = w.x < 0x80000000u;
+    if (threadIdx.x == 0 && keep) keep[b] = static_cast<uint8_t>(kept);
+    if (kept) return;
+    uint4* dst = reinterpret_cast<uint4*>(z + static_cast<int64_t>(b) * seq_elems);
+    const int64_t n = seq_elems / 8;
+    for (int64_t j = threadIdx.x; j < n; j += blockDim.x) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+}  // namespace
+
+cudaError_t launch_canvas_decide(const DecideParams& p, int32_t B, cudaStream_t s) {
+    if (B < 1 || p.C < 1 || p.C > DG_MAX_CANVAS_ROWS) return cudaErrorInvalidValue;
+    canvas_decide_kernel<<<B, kDecideThreads, 0, s>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ce_backward(const CeBackwardParams& p, cudaStream_t s) {
+    const int32_t vec_per_row = p.V / 8;
+    const dim3 grid(static_cast<unsigned>((vec_per_row + kCeVec * 256 - 1) / (kCeVec * 256)),
+                    static_cast<unsigned>(std::min<int32_t>(p.R, 65535)));
+    ce_backward_kernel<<<grid, 256, 0, s>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selfcond_drop(uint16_t* z, int32_t n_seq, int64_t seq_elems, uint32_t key0, uint32_t key1,
+                                 uint32_t step, uint8_t* keep, cudaStream_t s) {
+    selfcond_drop_kernel<<<n_seq, 256, 0, s>>>(z, seq_elems, key0, key1, step, keep);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace dg

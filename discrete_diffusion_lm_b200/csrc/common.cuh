@@ -30,6 +30,8 @@ enum : uint32_t {
     kDomNoise = 2,
     kDomCanvas = 3,
     kDomChunkGumbel = 4,
+    kDomRenoise = 5,  // entropy-bounded sampler: the re-noised token of a rejected position
+    kDomScDrop = 6,   // training: the self-conditioning keep/drop coin of a sequence
 };
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
@@ -82,6 +84,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Two floats rounded to nearest-even bf16, packed low/high.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

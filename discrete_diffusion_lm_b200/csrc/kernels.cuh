@@ -92,6 +92,46 @@ cudaError_t launch_bounded_wait_test(long long limit_cycles, cudaStream_t s);
 // Reads (synchronously) and clears the error word set by a kernel whose bounded wait expired.
 cudaError_t read_and_clear_device_error(int* out);
 
+// Per-canvas sampler decisions: entropy-bounded acceptance with uniform re-noising, and the
+// adaptive-stopping flag.  One CTA per canvas.  Null outputs skip their part (x_next == nullptr:
+// no acceptance; stop and mean_entropy both nullptr: no stopping test).
+struct DecideParams {
+    const float* entropy;        // [B*C]
+    const int32_t* x0_hat;       // [B*C]           (acceptance)
+    const int32_t* argmax;       // [B*C]           (stopping)
+    const int32_t* argmax_prev;  // [B*C] or null   (stopping; null: no previous step)
+    int32_t C, V;
+    long long accept_limit;      // accept while the rank-ordered prefix sum of q is below this
+    long long stop_limit;        // stop needs sum q below this
+    uint32_t key0, key1, step;
+    int32_t* x_next;             // [B*C]
+    uint8_t* accepted;           // [B*C] or null
+    int32_t* n_accepted;         // [B] or null
+    uint8_t* stop;               // [B] or null
+    float* mean_entropy;         // [B] or null
+};
+cudaError_t launch_canvas_decide(const DecideParams& p, int32_t B, cudaStream_t s);
+
+// Canvas cross-entropy gradient, in place over bf16 logits rows.
+struct CeBackwardParams {
+    void* logits;  // bf16 [R, ld], overwritten by the gradient
+    int64_t ld;
+    const float* lse;         // [R] saved by the forward pass
+    const int32_t* x0;        // [n_seq, seq_len]
+    const int32_t* canvas_idx;  // [n_seq]
+    const float* g_seq;       // [n_seq] upstream gradient of each sequence's summed loss, or null (1)
+    int32_t R, C, V, P, K;
+    int64_t seq_len;
+};
+cudaError_t launch_ce_backward(const CeBackwardParams& p, cudaStream_t s);
+
+// Zero the self-conditioning rows (C*d bf16 values per sequence) of sequences whose coin drops them.
+cudaError_t launch_selfcond_drop(uint16_t* z, int32_t n_seq, int64_t seq_elems, uint32_t key0, uint32_t key1,
+                                 uint32_t step, uint8_t* keep, cudaStream_t s);
+
+// Multiprocessor count of the current device (cached per device).
+int num_sms();
+
 // Count of kernels launched by the library (for the launch-count query).
 void note_launches(uint64_t n);
 

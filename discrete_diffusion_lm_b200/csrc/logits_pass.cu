@@ -170,15 +170,17 @@ struct MergeShared {
 };
 
 // Per-row merge, run by the last CTA of the row.  Global memory is visited in two round trips:
-// the chunk records (thread t holds the four consecutive chunks 4t .. 4t+3 in registers, so one
-// Philox call serves its four chunk Gumbel variates), then the two chunks that must be re-read
-// (the one holding the argmax and the level-1 winner), fetched together.  Rows of more than
-// 4 * kPassThreads chunks re-read their further records from L2 in each pass.
+// the chunk records (thread t holds quads of four consecutive chunks 4q .. 4q+3, q = t + u T, in
+// registers, so one Philox call serves four chunk Gumbel variates), then the two chunks that must
+// be re-read (the one holding the argmax and the level-1 winner), fetched together.
 //
 // Three block-wide exchanges: (1) the argmax over the chunk maxima and the level-1 winner, which
 // fixes both chunks to re-read, so their loads are in flight during (2) the log-sum-exp merge of
 // (S, T); (3) the argmax inside the argmax chunk and the level-2 winner.
-static_assert(kChunk == 4 * kPassThreads, "one chunk is re-read as four ids per thread");
+// A re-read chunk is kQuads quads of four consecutive ids per thread: ids lo + 4 (tid + u T) + k.
+constexpr int kQuads = kChunk / (4 * kPassThreads);
+constexpr int kRecQuads = (512 / 4 + kPassThreads - 1) / kPassThreads;
+static_assert(kQuads >= 1 && kChunk == 4 * kQuads * kPassThreads, "a chunk splits into whole quads per thread");
 
 template <bool kBf16, int kKind>
 __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t canvas, float inv_tau,
@@ -190,7 +192,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 
     // Scalars needed at the very end, loaded first so their latency overlaps the merge.
     int32_t xt = 0;
-    if (kKind == kPassSampler && tid == 0) xt = p.x_t[row];
+    if (kKind == kPassSampler && tid == 0 && p.x_t) xt = p.x_t[row];
     float target_logit = 0.f;
     bool target_ok = false;
     int32_t b_seq = 0, i_seq = 0;
@@ -208,13 +210,17 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         }
     }
 
-    float4 r[4];
+    // Quads q = tid + u T (u < kRecQuads) stay in registers: all records of rows up to 512 chunks.
+    float4 r[kRecQuads][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int32_t j = 4 * tid + k;
-        r[k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
-    }
-    // Records beyond the first 4 * kPassThreads (rows longer than 262144 ids with 128 threads).
+    for (int u = 0; u < kRecQuads; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int32_t j = 4 * (tid + u * kPassThreads) + k;
+            r[u][k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        }
+    // Records beyond those (rows longer than 262144 ids) are re-read from L2 in each pass.
+    constexpr int kFar = kRecQuads * kPassThreads;
     auto far_quad = [&](int32_t q, float4 (&f)[4]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -252,8 +258,10 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             }
         }
     };
-    if (4 * tid < nch) scan_quad(tid, r);
-    for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
+#pragma unroll
+    for (int u = 0; u < kRecQuads; ++u)
+        if (4 * (tid + u * kPassThreads) < nch) scan_quad(tid + u * kPassThreads, r[u]);
+    for (int32_t q = tid + kFar; 4 * q < nch; q += kPassThreads) {
         float4 f[4];
         far_quad(q, f);
         scan_quad(q, f);
@@ -265,16 +273,18 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const float m_row = m_raw * inv_tau;
 
     // Both re-read chunks are known: ids lo + 4 tid .. lo + 4 tid + 3 of each, loaded now.
-    float av[4], gv[4];
+    float av[kQuads][4], gv[kQuads][4];
     const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
     const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
     if (kKind == kPassSampler) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int32_t va = alo + 4 * tid + k, vg = glo + 4 * tid + k;
-            av[k] = va < ahi ? fmaxf(load_logit(rowp, va, kBf16), nbig) : -INFINITY;
-            gv[k] = vg < ghi ? fmaxf(load_logit(rowp, vg, kBf16), nbig) : -INFINITY;
-        }
+        for (int u = 0; u < kQuads; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int32_t o = 4 * (tid + u * kPassThreads) + k;
+                av[u][k] = alo + o < ahi ? fmaxf(load_logit(rowp, alo + o, kBf16), nbig) : -INFINITY;
+                gv[u][k] = glo + o < ghi ? fmaxf(load_logit(rowp, glo + o, kBf16), nbig) : -INFINITY;
+            }
     }
 
     // (2) Log-sum-exp merge of (S, T) relative to the row maximum.
@@ -287,8 +297,10 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         t = fmaf(f, fmaf(c.y, dm, c.z), t);
     };
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc_st(r[k]);
-    for (int32_t q = tid + kPassThreads; 4 * q < nch; q += kPassThreads) {
+    for (int u = 0; u < kRecQuads; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc_st(r[u][k]);
+    for (int32_t q = tid + kFar; 4 * q < nch; q += kPassThreads) {
         float4 f[4];
         far_quad(q, f);
 #pragma unroll
@@ -339,25 +351,30 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     float amv = -INFINITY;
     int am = 0x7fffffff;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-        if (av[k] > amv) {
-            amv = av[k];
-            am = alo + 4 * tid + k;
-        }
+    for (int u = 0; u < kQuads; ++u)  // ascending ids, strict: the first maximum wins
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (av[u][k] > amv) {
+                amv = av[u][k];
+                am = alo + 4 * (tid + u * kPassThreads) + k;
+            }
     float bs2 = -INFINITY;
     int bv = 0x7fffffff;
-    const int32_t vg0 = glo + 4 * tid;
-    if (sampling && vg0 < ghi) {
-        const uint4 w = philox4x32_10(
-            make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel), p.key0,
-            p.key1);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if (vg0 + k < ghi) {
-                const float sc = gv[k] * inv_tau + gumbel_from_word(word_of(w, k));
-                if (sc > bs2) {
-                    bs2 = sc;
-                    bv = vg0 + k;
+    for (int u = 0; u < kQuads; ++u) {
+        const int32_t vg0 = glo + 4 * (tid + u * kPassThreads);
+        if (sampling && vg0 < ghi) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
+                p.key0, p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (vg0 + k < ghi) {
+                    const float sc = gv[u][k] * inv_tau + gumbel_from_word(word_of(w, k));
+                    if (sc > bs2) {
+                        bs2 = sc;
+                        bv = vg0 + k;
+                    }
                 }
             }
         }
@@ -367,41 +384,44 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const int32_t x0 = sampling && bv >= glo && bv < ghi ? bv : am;
 
     if (tid == 0) {
-        unsigned long long t_stay, t_jump;
-        if (x0 != xt) {
-            t_stay = p.thr_stay_diff[canvas];
-            t_jump = p.thr_jump_diff[canvas];
-        } else {
-            t_stay = p.thr_stay_same[canvas];
-            t_jump = t_stay;
+        if (p.x_next) {  // the Step posterior (skipped when a per-canvas rule decides instead)
+            unsigned long long t_stay, t_jump;
+            if (x0 != xt) {
+                t_stay = p.thr_stay_diff[canvas];
+                t_jump = p.thr_jump_diff[canvas];
+            } else {
+                t_stay = p.thr_stay_same[canvas];
+                t_jump = t_stay;
+            }
+            const uint4 w =
+                philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), p.step, kDomStep), p.key0, p.key1);
+            const unsigned long long u = w.x;
+            int32_t xn;
+            uint8_t br;
+            if (u < t_stay) {
+                xn = xt;
+                br = 0;
+            } else if (u < t_jump) {
+                xn = x0;
+                br = 1;
+            } else {
+                xn = word_to_index(w.y, p.V);
+                br = 2;
+            }
+            p.x_next[row] = xn;
+            if (p.branch) p.branch[row] = br;
         }
-        const uint4 w = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), p.step, kDomStep), p.key0, p.key1);
-        const unsigned long long u = w.x;
-        int32_t xn;
-        uint8_t br;
-        if (u < t_stay) {
-            xn = xt;
-            br = 0;
-        } else if (u < t_jump) {
-            xn = x0;
-            br = 1;
-        } else {
-            xn = word_to_index(w.y, p.V);
-            br = 2;
-        }
-        p.x_next[row] = xn;
         if (p.x0_hat) p.x0_hat[row] = x0;
         if (p.argmax) p.argmax[row] = am;
         if (p.max_prob) p.max_prob[row] = 1.0f / S;
         if (p.lse) p.lse[row] = lse;
         if (p.entropy) p.entropy[row] = ln_s - T / S;
-        if (p.branch) p.branch[row] = br;
         p.row_ticket[row] = 0u;
     }
 }
 
 template <bool kBf16, int kKind>
-__global__ void __launch_bounds__(kPassThreads) logits_pass_kernel(const __grid_constant__ PassParams p) {
+__global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kernel(const __grid_constant__ PassParams p) {
     __shared__ MergeShared sh;
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;

@@ -164,11 +164,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 // p for 8 consecutive bf16 logits held in one 16-byte chunk, packed back as 8 bf16.
 __device__ __forceinline__ uint4 softmax_chunk_bf16(uint4 c, float a, float nb) {
     uint4 o;
@@ -795,17 +790,6 @@ int pick_ntile(int d, bool logits_bf16) {
     return logits_bf16 ? nt : (nt > 256 ? 256 : nt);
 }
 
-int num_sms() {
-    static std::atomic<int> cached{0};
-    int v = cached.load();
-    if (v == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-        cached.store(v);
-    }
-    return v;
-}
 
 // Work plan: CTA pairs (M = 256 per pair) when there are more than 128 rows and the column tile
 // is at least 128 wide, single CTAs otherwise; the vocabulary is split so that the grid is about
@@ -865,6 +849,18 @@ cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st
 }
 
 }  // namespace
+
+int num_sms() {
+    static std::atomic<int> cached{0};
+    int v = cached.load();
+    if (v == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cached.store(v);
+    }
+    return v;
+}
 
 size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16) {
     if (R < 1 || V < 1 || d < 64) return 0;

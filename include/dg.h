@@ -82,6 +82,7 @@ typedef enum dg_x0_mode { DG_X0_SAMPLE = 0, DG_X0_GREEDY = 1 } dg_x0_mode;
 
 #define DG_GUMBEL_CHUNK 512
 #define DG_MAX_CANVASES 256 /* canvases (B, n_seq) per call */
+#define DG_MAX_CANVAS_ROWS 1024 /* C for the per-canvas decisions (acceptance, stopping) */
 
 /* Human-readable reason for the last failure on this thread ("" if none). */
 const char* dg_last_error(void);
@@ -175,6 +176,94 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
                  size_t workspace_bytes, dg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Temperature schedule (section "Method", sampler paragraph: tau_t < 1 is  */
+/* annealed linearly over the denoising time scale from tau_max = 0.8 to    */
+/* tau_min = 0.4).  Host only: inv_tau[b] = 1 / (tau_min + (tau_max -       */
+/* tau_min) clamp(t[b], 0, 1)), ready for the inv_tau arguments above.      */
+/* t: host double [B] (not NaN); inv_tau: host float [B].  tau_max, tau_min */
+/* finite and > 0.  Returns DG_ERR_INVALID_ARG otherwise.                   */
+/* ------------------------------------------------------------------------ */
+int dg_tau_linear(const double* t, int32_t B, double tau_max, double tau_min, float* inv_tau);
+
+/* ------------------------------------------------------------------------ */
+/* Entropy-bounded acceptance (section "Method", sampler paragraph: tokens  */
+/* are accepted in ascending order of entropy while an error bound stays    */
+/* strictly below a tolerance; every other token is re-noised uniformly at  */
+/* random).  Per canvas b of C rows r = b*C + i:                            */
+/*   q_i = floor(clamp(entropy[r], 0, 64) 2^32)   (NaN counts as 64)        */
+/*   order the rows by ascending (q_i, i); the k-th of that order is        */
+/*   accepted iff q_(1) + ... + q_(k) < ceil(eps 2^32)                      */
+/*   x_next[r] = accepted ? x0_hat[r] : floor(w0 V / 2^32),                 */
+/*   w0 = Philox4x32-10(counter (0, r, step, 5), key seed) word 0.          */
+/* The bound of an accepted set is read as the sum of its entropies (an     */
+/* upper bound on its total correlation); the pages give no formula.        */
+/* entropy: device float [B*C]; x0_hat: device int32 [B*C].                 */
+/* Outputs (device): x_next int32 [B*C] (required), accepted uint8 [B*C]     */
+/* and n_accepted int32 [B] (each may be NULL).  1 <= B <= DG_MAX_CANVASES, */
+/* 1 <= C <= DG_MAX_CANVAS_ROWS (DG_ERR_UNSUPPORTED above), eps not NaN.    */
+/* One CTA per canvas, no workspace.                                        */
+/* ------------------------------------------------------------------------ */
+int dg_entropy_accept(const float* entropy, const int32_t* x0_hat, int32_t B, int32_t C, int32_t V,
+                      double eps, uint64_t seed, uint32_t step, int32_t* x_next, uint8_t* accepted,
+                      int32_t* n_accepted, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive stopping (section "Method", sampler paragraph: stop when the    */
+/* canvas-mean predicted entropy is below a threshold and the deterministic */
+/* predictions of two consecutive steps are identical).  Per canvas b:      */
+/*   stop[b] = sum_i q_i < ceil(theta C 2^32)  and  argmax == argmax_prev   */
+/*             at every row of the canvas (q as in dg_entropy_accept);      */
+/*   mean_entropy[b] = float((double) sum_i q_i 2^-32 / C).                 */
+/* argmax, argmax_prev: device int32 [B*C]; argmax_prev NULL = no previous  */
+/* step (stop is then 0).  Outputs device: stop uint8 [B], mean_entropy     */
+/* float [B]; at least one non-NULL.  Limits as dg_entropy_accept.          */
+/* ------------------------------------------------------------------------ */
+int dg_adaptive_stop(const float* entropy, const int32_t* argmax, const int32_t* argmax_prev,
+                     int32_t B, int32_t C, double theta, uint8_t* stop, float* mean_entropy,
+                     dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Entropy-bounded sampler step: the statistics, argmax and x0_hat draw of  */
+/* dg_sampler_step (its Step posterior is not applied), then the            */
+/* acceptance and stopping decisions above on the step's own entropy and    */
+/* argmax.  Two launches on `stream`.  Arguments as dg_sampler_step and the */
+/* two functions above; x_next, x0_hat and entropy are required, argmax is  */
+/* required when stop or mean_entropy is requested.  Workspace: the size   */
+/* dg_sampler_step_workspace_size(B*C, V) gives, same contract.            */
+/* ------------------------------------------------------------------------ */
+int dg_sampler_step_eb(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C,
+                       int32_t V, const float* inv_tau, uint64_t seed, uint32_t step, int x0_mode,
+                       double eps, double theta, const int32_t* argmax_prev, int32_t* x_next,
+                       int32_t* x0_hat, int32_t* argmax, float* max_prob, float* lse,
+                       float* entropy, uint8_t* accepted, uint8_t* stop, float* mean_entropy,
+                       void* workspace, size_t workspace_bytes, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Canvas cross-entropy backward (section "Method", loss equation): for row */
+/* r = b*C + i with target y = x0[b, P + canvas_idx[b]*C + i],               */
+/*   logits[r, v] <- g_seq[b] (exp(logits[r, v] - lse_rows[r]) - [v == y])  */
+/* in place, rounded to bf16; rows whose target (or canvas index) is out of */
+/* range become zero.  logits: device bf16 [n_seq*C, ld], V and ld multiples*/
+/* of 8, 16-byte aligned.  lse_rows: device float [n_seq*C] as dg_canvas_ce */
+/* writes it.  g_seq: device float [n_seq] (the upstream gradient of each   */
+/* sequence's summed loss) or NULL for 1.  No workspace.                    */
+/* ------------------------------------------------------------------------ */
+int dg_canvas_ce_backward(void* logits, int64_t ld, const float* lse_rows, const int32_t* x0,
+                          const int32_t* canvas_idx, int32_t n_seq, int32_t P, int32_t K,
+                          int32_t C, int32_t V, const float* g_seq, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Self-conditioning drop for training (section "Dataset": for half of the  */
+/* batch the decoder uses the previous pass's self-conditioning state, for  */
+/* the other half that state is zero).  keep[b] = w0 < 2^31 with w0 from    */
+/* Philox4x32-10(counter (0, b, step, 6), key seed); the C*d bf16 values of */
+/* a dropped sequence are set to zero in place.  z: device bf16 [n_seq*C, d]*/
+/* 16-byte aligned, C*d a multiple of 8.  keep: device uint8 [n_seq] or NULL.*/
+/* ------------------------------------------------------------------------ */
+int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed, uint32_t step,
+                     uint8_t* keep, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Failure-detection test hooks (the pages have no counterpart).  Every wait */
 /* inside the library's kernels is bounded; these entry points make a wait  */
 /* run out on purpose -- without any fault, trap or endless loop -- so that */
@@ -182,8 +271,8 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
 /* dg_device_error() (code 1) and leaves the device usable.                 */
 /* dg_test_bounded_wait: one thread waits on a barrier nothing arrives on;  */
 /*   the wait gives up after limit_cycles (> 0) SM clock cycles.             */
-/* dg_test_selfcond_stall: dg_selfcond with the copy of one 32-id block of  */
-/*   E never issued (stalled_block >= 0, in [0, ceil(V/32)) to take effect) */
+/* dg_test_selfcond_stall: dg_selfcond with the copy of one 64-id block of  */
+/*   E never issued (stalled_block >= 0, in [0, ceil(V/64)) to take effect) */
 /*   and every wait limited to limit_cycles: the CTAs that need the block   */
 /*   abort, drain their in-flight copies, free their tensor memory and      */
 /*   return.  z is then incomplete.  Same arguments as dg_selfcond otherwise.*/

@@ -126,3 +126,39 @@ def test_workspace_queries(L):
     assert dg.dg_canvas_ce_workspace_size(8, 256, 262144) >= 2048 * 128 * 16
     assert dg.dg_selfcond_workspace_size(256, 262144, 2048, 1, 1, True) >= 0
     assert dg.dg_selfcond_workspace_size(256, 262144, 2048, 1, 0, True) >= 262144 * 2048 * 2
+
+
+def test_sampler_extensions_reject(L):
+    ea = L.dg_entropy_accept
+    assert ea(None, FAKE, 1, 16, 100, ctypes.c_double(1.0), 0, 0, FAKE, None, None, None) == 1
+    assert ea(FAKE, FAKE, 1, 16, 100, ctypes.c_double(1.0), 0, 0, None, None, None, None) == 1
+    assert ea(FAKE, FAKE, 1, 1025, 100, ctypes.c_double(1.0), 0, 0, FAKE, None, None, None) == 5  # C > max
+    assert ea(FAKE, FAKE, 0, 16, 100, ctypes.c_double(1.0), 0, 0, FAKE, None, None, None) == 1
+    assert ea(FAKE, FAKE, 1, 16, 100, ctypes.c_double(float("nan")), 0, 0, FAKE, None, None, None) == 1
+    st = L.dg_adaptive_stop
+    assert st(FAKE, FAKE, None, 1, 16, ctypes.c_double(0.5), None, None, None) == 1  # no output
+    assert st(FAKE, None, None, 1, 16, ctypes.c_double(0.5), FAKE, None, None) == 1
+    eb = L.dg_sampler_step_eb
+    args = [FAKE, 1, 1024, 1, 16, 1024, None, 0, 0, 0, ctypes.c_double(1.0), ctypes.c_double(0.5), None,
+            FAKE, FAKE, None, None, None, FAKE, None, FAKE, None, FAKE, 1 << 30, None]
+    assert eb(*args) == 1  # stop requested without argmax
+    a2 = list(args)
+    a2[20] = None
+    a2[13] = None
+    assert eb(*a2) == 1  # x_next missing
+    bw = L.dg_canvas_ce_backward
+    assert bw(FAKE, 1028, FAKE, FAKE, FAKE, 2, 4, 2, 8, 1028, None, None) == 2  # V not a multiple of 8
+    assert bw(FAKE, 1024, None, FAKE, FAKE, 2, 4, 2, 8, 1024, None, None) == 1
+    dr = L.dg_selfcond_drop
+    assert dr(FAKE + 8, 2, 4, 8, 0, 0, None, None) == 2
+    assert dr(FAKE, 2, 3, 3, 0, 0, None, None) == 2  # C*d not a multiple of 8
+
+
+def test_tau_linear_host_matches_oracle(L):
+    from oracle import oracle as O
+    ts = [0.0, 0.1, 0.5, 0.73, 1.0, -0.5, 1.5]
+    got = dg.dg_tau_linear(ts)
+    for t, g in zip(ts, got):
+        assert g == pytest.approx(1.0 / O.tau_linear(t), rel=1e-7)
+    out = (ctypes.c_float * 1)()
+    assert L.dg_tau_linear((ctypes.c_double * 1)(0.5), 1, ctypes.c_double(0.8), ctypes.c_double(0.0), out) == 1
