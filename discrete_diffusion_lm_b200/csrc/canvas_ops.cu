@@ -16,7 +16,8 @@
 //   accepted set is the ranks whose prefix is below the tolerance.  Stopping: the sum of q
 //   against the threshold, and an all-equal test of the argmax canvas against the previous one.
 // ce_backward_kernel: rows along grid y, 16-byte bf16 vectors of a row along grid x, in place.
-// selfcond_drop_kernel: one CTA per sequence; a fair Philox coin decides, dropped rows are zeroed.
+// selfcond_drop_kernel: sequences along grid y; a fair Philox coin per sequence decides, dropped
+//   rows are zeroed.
 #include <algorithm>
 
 #include "common.cuh"
@@ -197,16 +198,19 @@ __global__ void __launch_bounds__(256) ce_backward_kernel(const __grid_constant_
     }
 }
 
+// Grid: y = sequence, x = 4 KB slices of its C*d values (256 threads x one 16-byte vector).
 __global__ void __launch_bounds__(256) selfcond_drop_kernel(uint16_t* z, int64_t seq_elems, uint32_t key0,
                                                             uint32_t key1, uint32_t step, uint8_t* keep) {
-    const int b = blockIdx.x;
+    const int b = blockIdx.y;
     const uint4 w = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(b), step, kDomScDrop), key0, key1);
     const bool kept = w.x < 0x80000000u;
-    if (threadIdx.x == 0 && keep) keep[b] = static_cast<uint8_t>(kept);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && keep) keep[b] = static_cast<uint8_t>(kept);
     if (kept) return;
     uint4* dst = reinterpret_cast<uint4*>(z + static_cast<int64_t>(b) * seq_elems);
     const int64_t n = seq_elems / 8;
-    for (int64_t j = threadIdx.x; j < n; j += blockDim.x) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        dst[j] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace
@@ -229,7 +233,9 @@ cudaError_t launch_ce_backward(const CeBackwardParams& p, cudaStream_t s) {
 
 cudaError_t launch_selfcond_drop(uint16_t* z, int32_t n_seq, int64_t seq_elems, uint32_t key0, uint32_t key1,
                                  uint32_t step, uint8_t* keep, cudaStream_t s) {
-    selfcond_drop_kernel<<<n_seq, 256, 0, s>>>(z, seq_elems, key0, key1, step, keep);
+    const int64_t n = seq_elems / 8;
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 1024)), static_cast<unsigned>(n_seq));
+    selfcond_drop_kernel<<<grid, 256, 0, s>>>(z, seq_elems, key0, key1, step, keep);
     note_launches(1);
     return cudaGetLastError();
 }
