@@ -170,3 +170,18 @@ def make_train_logits(cfg: TrainConfig, device="cpu", rows: int | None = None) -
         out[r0:r1] = (torch.randn((r1 - r0, cfg.V), generator=g, device=device) * cfg.logits_std).to(
             torch.bfloat16)
     return out
+
+
+# Feed-forward block on the self-conditioning input: hidden width = FFW_RATIO x d.
+FFW_RATIO = 4
+
+
+def make_ffw(cfg: SamplerConfig, device="cpu", seed: int | None = None):
+    """Random-init weights of the two-layer feed-forward block and a self-conditioning input:
+    z ~ N(0, 1) [R, d], W1 ~ N(0, 1/d) [d, 4d], W2 ~ N(0, 1/(4d)) [4d, d], all bf16."""
+    s = cfg.seed if seed is None else seed
+    dff = FFW_RATIO * cfg.d
+    z = torch.randn(cfg.R, cfg.d, generator=_gen(device, s + 600), device=device)
+    w1 = torch.randn(cfg.d, dff, generator=_gen(device, s + 700), device=device) * cfg.d ** -0.5
+    w2 = torch.randn(dff, cfg.d, generator=_gen(device, s + 800), device=device) * dff ** -0.5
+    return z.to(torch.bfloat16), w1.to(torch.bfloat16), w2.to(torch.bfloat16)

@@ -633,3 +633,42 @@ void dgo_selfcond_drop(double* z, int32_t n_seq, int32_t C, int32_t d, uint64_t 
             for (int64_t j = (int64_t)b * C * d; j < ((int64_t)b + 1) * C * d; ++j) z[j] = 0.0;
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Feed-forward block on the self-conditioning input [TR-Method:            */
+/* z = FFW(p0 E), FFW a standard feed-forward network].  Reading (the pages */
+/* name no architecture and no trained weights exist): a two-layer          */
+/* perceptron without biases, out = gelu(z W1) W2, with the tanh form of    */
+/* GELU (Hendrycks and Gimpel, "Gaussian Error Linear Units", 2016):        */
+/*     gelu(x) = x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).             */
+/* z [R, d], W1 [d, dff], W2 [dff, d] row-major (float, widened from bf16   */
+/* by the caller); out [R, d] in double, no rounding between the layers.    */
+/* ------------------------------------------------------------------------ */
+double dgo_gelu_tanh(double x)
+{
+    const double k = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * x * (1.0 + tanh(k * (x + 0.044715 * x * x * x)));
+}
+
+void dgo_ffw(const float* z, const float* W1, const float* W2, int32_t R, int32_t d, int32_t dff,
+             double* out)
+{
+    double* h = (double*)malloc(sizeof(double) * (size_t)dff);
+    for (int32_t r = 0; r < R; ++r) {
+        for (int32_t j = 0; j < dff; ++j) h[j] = 0.0;
+        for (int32_t k = 0; k < d; ++k) {
+            double zk = (double)z[(int64_t)r * d + k];
+            const float* w = W1 + (int64_t)k * dff;
+            for (int32_t j = 0; j < dff; ++j) h[j] += zk * (double)w[j];
+        }
+        for (int32_t j = 0; j < dff; ++j) h[j] = dgo_gelu_tanh(h[j]);
+        double* o = out + (int64_t)r * d;
+        for (int32_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int32_t j = 0; j < dff; ++j) {
+            double hj = h[j];
+            const float* w = W2 + (int64_t)j * d;
+            for (int32_t c = 0; c < d; ++c) o[c] += hj * (double)w[c];
+        }
+    }
+    free(h);
+}

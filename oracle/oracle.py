@@ -81,6 +81,9 @@ def _declare(L):
     L.dgo_adaptive_stop.argtypes = [_p, _p, _p, _i32, _i32, _f64, _p, _p]
     L.dgo_canvas_ce_backward.argtypes = [_p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p]
     L.dgo_selfcond_drop.argtypes = [_p, _i32, _i32, _i32, _u64, _u32, _p]
+    L.dgo_gelu_tanh.argtypes = [_f64]
+    L.dgo_gelu_tanh.restype = _f64
+    L.dgo_ffw.argtypes = [_p, _p, _p, _i32, _i32, _i32, _p]
 
 
 def _ptr(a: np.ndarray):
@@ -269,3 +272,18 @@ def selfcond_drop(z, n_seq: int, C: int, d: int, seed: int, step: int):
     keep = np.zeros(n_seq, dtype=np.uint8)
     lib().dgo_selfcond_drop(_ptr(zz), n_seq, C, d, seed, step, _ptr(keep))
     return zz, keep
+
+
+def gelu_tanh(x: float) -> float:
+    return lib().dgo_gelu_tanh(float(x))
+
+
+def ffw(z, W1, W2) -> np.ndarray:
+    """Two-layer feed-forward block gelu(z W1) W2 in double: z [R, d], W1 [d, dff], W2 [dff, d]."""
+    zz, a, b = _f32(z), _f32(W1), _f32(W2)
+    R, d = zz.shape
+    dff = a.shape[1]
+    assert a.shape == (d, dff) and b.shape == (dff, d)
+    out = np.zeros((R, d), dtype=np.float64)
+    lib().dgo_ffw(_ptr(zz), _ptr(a), _ptr(b), R, d, dff, _ptr(out))
+    return out

@@ -193,3 +193,27 @@ def test_selfcond_drop_fair_coin_and_zeroing():
     assert (zz[keep == 1] == z0[keep == 1]).all()
     _, keep2 = O.selfcond_drop(z, n_seq, C, d, 9, 1)
     assert 0.4 < (keep2 != keep).mean() < 0.6  # a new coin per step
+
+
+# ----------------------------------------------------------------------------- FFW
+def test_gelu_tanh_against_torch_and_limits():
+    xs = np.linspace(-8, 8, 161)
+    ref = torch.nn.functional.gelu(torch.tensor(xs, dtype=torch.float64), approximate="tanh").numpy()
+    got = np.array([O.gelu_tanh(x) for x in xs])
+    assert np.allclose(got, ref, rtol=1e-14, atol=1e-15)
+    assert O.gelu_tanh(0.0) == 0.0
+    assert O.gelu_tanh(30.0) == pytest.approx(30.0) and abs(O.gelu_tanh(-30.0)) < 1e-30
+
+
+def test_ffw_against_torch_float64():
+    rng = np.random.default_rng(2)
+    R, d, dff = 5, 16, 48
+    z = rng.standard_normal((R, d)).astype(np.float32)
+    W1 = (rng.standard_normal((d, dff)) / 4).astype(np.float32)
+    W2 = (rng.standard_normal((dff, d)) / 7).astype(np.float32)
+    got = O.ffw(z, W1, W2)
+    t = lambda a: torch.tensor(a, dtype=torch.float64)
+    ref = (torch.nn.functional.gelu(t(z) @ t(W1), approximate="tanh") @ t(W2)).numpy()
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-14)
+    assert np.allclose(O.ffw(np.zeros_like(z), W1, W2), 0.0)
+    assert np.allclose(O.ffw(z, W1, 2 * W2), 2 * got, rtol=1e-13)  # linear in the second layer
