@@ -278,6 +278,7 @@ def run_ours(args, rank, world, local):
     # ---- training-side kernels on the training workload (forward noise + canvas CE + backward)
     train = bench_train(dg, W, dev, stream, hbm)
     eb = bench_eb(dg, W, dev, stream, bufs, hbm)
+    ffw = bench_ffw(dg, W, dev, stream, peaks)
 
     # ---- end to end through the public API with host buffers
     e2e = bench_e2e(dg, W, cfg, dev, E, args, world, barrier)
@@ -311,6 +312,7 @@ def run_ours(args, rank, world, local):
             "selfcond_frac_hbm": round(bytes_k2 / (k2_mean * 1e-6) / 1e9 / hbm, 4),
             "train": train,
             "entropy_bounded": eb,
+            "ffw": ffw,
         },
         "e2e": e2e,
         "gpu_launches": int(round(launches_per_step * K)),
@@ -397,6 +399,39 @@ def bench_train(dg, W, dev, stream, hbm):
             "ce_backward_frac_hbm": round(bw_bytes / (bw_us * 1e-6) / 1e9 / hbm, 4),
             "selfcond_drop_us": round(drop_us, 2),
             "note": "canvas CE logits (1.07 GB) exceed L2; repeated on one buffer (the backward in place)"}
+
+
+def bench_ffw(dg, W, dev, stream, peaks):
+    """The feed-forward block on the self-conditioning input at the full size (R=256, d=2048,
+    d_ff=8192, random bf16 weights): both layers, each a tcgen05 contraction + split sum."""
+    import torch
+    cfg = W.FULL
+    z, w1, w2 = W.make_ffw(cfg, dev)
+    out, hidden = dg.dg_ffw(z, w1, w2, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        dg.dg_ffw(z, w1, w2, hidden=hidden, out=out, stream=stream)
+    reps = 50
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            g.replay()
+        e[0].record(stream)
+        for _ in range(reps):
+            g.replay()
+        e[1].record(stream)
+    stream.synchronize()
+    us = e[0].elapsed_time(e[1]) * 1e3 / reps
+    dff = W.FFW_RATIO * cfg.d
+    flops = 2.0 * 2 * cfg.R * cfg.d * dff
+    nbytes = 2 * cfg.d * dff * 2 + cfg.R * (2 * cfg.d + 2 * dff) * 2
+    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    bound_us = max(flops / (tc * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+    return {"workload": f"FFW gelu(z W1) W2: R={cfg.R}, d={cfg.d}, d_ff={dff}, bf16, weights {nbytes / 1e6:.0f} MB "
+                        "(L2-resident across replays)",
+            "ffw_us": round(us, 2), "ffw_TFLOPs": round(flops / (us * 1e-6) / 1e12, 1),
+            "ffw_frac_of_slower_bound": round(bound_us / us, 4), "slower_bound_us": round(bound_us, 2)}
 
 
 def bench_eb(dg, W, dev, stream, bufs, hbm):

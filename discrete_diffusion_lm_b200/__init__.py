@@ -74,6 +74,9 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_double, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]
         L.dg_canvas_ce_backward.argtypes = [_p, _i64, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p]
         L.dg_selfcond_drop.argtypes = [_p, _i32, _i32, _i32, _u64, _u32, _p, _p]
+        L.dg_ffw_workspace_size.argtypes = [_i32, _i32, _i32]
+        L.dg_ffw_workspace_size.restype = _sz
+        L.dg_ffw.argtypes = [_p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]
         _lib = L
     return _lib
 
@@ -427,3 +430,26 @@ def dg_selfcond_drop(z: torch.Tensor, C: int, *, seed: int = 0, step: int = 0,
                                 _stream(stream))
     _check("dg_selfcond_drop", rc)
     return keep
+
+
+def dg_ffw(z: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, *, hidden: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Two-layer feed-forward block gelu(z W1) W2 on the tensor cores (bf16 in and out).
+    Returns (out [R, d], hidden [R, d_ff])."""
+    for t, n in ((z, "z"), (W1, "W1"), (W2, "W2")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bf16 tensor")
+    R, d = z.shape
+    dff = W1.shape[1]
+    if W1.shape != (d, dff) or W2.shape != (dff, d):
+        raise ValueError("W1 must be [d, d_ff] and W2 [d_ff, d]")
+    dev = z.device
+    hidden = torch.empty(R, dff, dtype=torch.bfloat16, device=dev) if hidden is None else hidden
+    out = torch.empty(R, d, dtype=torch.bfloat16, device=dev) if out is None else out
+    nbytes = int(lib().dg_ffw_workspace_size(R, d, dff))
+    if ws is None:
+        ws = workspace("ffw", nbytes, dev, (R, d, dff), stream)
+    rc = lib().dg_ffw(_ptr(z), R, d, dff, _ptr(W1), _ptr(W2), _ptr(hidden), _ptr(out), _ptr(ws),
+                      ws.numel() * ws.element_size(), _stream(stream))
+    _check("dg_ffw", rc)
+    return out, hidden

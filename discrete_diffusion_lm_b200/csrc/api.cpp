@@ -660,4 +660,55 @@ int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed
     return DG_OK;
 }
 
+
+size_t dg_ffw_workspace_size(int32_t rows, int32_t d, int32_t d_ff) {
+    if (rows < 1 || d < 64 || d_ff < 64) return 0;
+    const size_t a = selfcond_partial_bytes(rows, d, d_ff, true);   // layer 1: K = d, N = d_ff
+    const size_t b = selfcond_partial_bytes(rows, d_ff, d, true);   // layer 2: K = d_ff, N = d
+    return a > b ? a : b;
+}
+
+int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* W1, const void* W2, void* hidden,
+           void* z_out, void* workspace, size_t workspace_bytes, dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if (!z_in || !W1 || !W2 || !hidden || !z_out)
+        return fail(DG_ERR_INVALID_ARG, "z_in, W1, W2, hidden and z_out are required");
+    if (rows < 1) return fail(DG_ERR_INVALID_ARG, "rows = %d must be >= 1", rows);
+    if (d < 64 || d > 16384 || d % 64 != 0 || d_ff < 64 || d_ff > 16384 || d_ff % 64 != 0)
+        return fail(DG_ERR_INVALID_ARG, "d = %d and d_ff = %d must be multiples of 64 in [64, 16384]", d, d_ff);
+    if (!aligned16(z_in) || !aligned16(W1) || !aligned16(W2) || !aligned16(hidden) || !aligned16(z_out))
+        return fail(DG_ERR_ALIGNMENT, "all operands must be 16-byte aligned");
+    if (z_in == z_out || hidden == z_in || hidden == z_out)
+        return fail(DG_ERR_INVALID_ARG, "z_in, hidden and z_out may not alias");
+    const size_t need = dg_ffw_workspace_size(rows, d, d_ff);
+    if (need && (!workspace || workspace_bytes < need))
+        return fail(DG_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+    if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(DG_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    if ((rc = check_device()) != DG_OK) return rc;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    static thread_local SelfcondParams sp;
+    for (int layer = 0; layer < 2; ++layer) {
+        std::memset(&sp, 0, sizeof(sp));
+        sp.logits = layer == 0 ? z_in : hidden;
+        sp.ld = layer == 0 ? d : d_ff;
+        sp.logits_bf16 = 1;
+        sp.E = static_cast<const uint16_t*>(layer == 0 ? W1 : W2);
+        sp.z = static_cast<uint16_t*>(layer == 0 ? hidden : z_out);
+        sp.R = rows;
+        sp.C = rows;
+        sp.V = layer == 0 ? d : d_ff;
+        sp.d = layer == 0 ? d_ff : d;
+        sp.partial = static_cast<float*>(workspace);
+        sp.fault_block = -1;
+        sp.plain_a = 1;
+        sp.act = layer == 0 ? 1 : 0;
+        sp.inv_tau[0] = 1.0f;
+        const cudaError_t e = launch_selfcond(sp, s);
+        if (e != cudaSuccess) return cuda_fail(e, layer == 0 ? "FFW layer 1 launch" : "FFW layer 2 launch");
+    }
+    return DG_OK;
+}
+
 }  // extern "C"

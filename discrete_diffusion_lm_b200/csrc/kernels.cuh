@@ -80,7 +80,9 @@ struct SelfcondParams {
     float* partial;      // fp32 [splits, R, d] (when the vocabulary is split)
     int32_t R, C, V, d;
     long long wait_limit;  // cycles before a stalled wait aborts the CTA (0: the library default)
-    int32_t fault_block;   // test hook: never issue the E copy of this 32-id block (-1: none)
+    int32_t fault_block;   // test hook: never issue the E copy of this 64-id block (-1: none)
+    int32_t plain_a;       // 1: `logits` is a plain bf16 A operand [R, V] (no softmax, lse unused)
+    int32_t act;           // epilogue activation on z: 0 none, 1 GELU (tanh form)
     float inv_tau[DG_MAX_CANVASES];
 };
 

@@ -51,8 +51,25 @@ struct alignas(64) KernelParams {
     int32_t n_tiles, splits, total_kb;
     long long wait_limit;  // cycles a wait may last before the CTA aborts
     int32_t fault_block;   // test hook: the E copy of this kKBlock-id block is never issued (-1: none)
+    int32_t plain;         // 1: the A tiles are the bf16 operand as loaded (no softmax; lse unused)
+    int32_t act;           // epilogue activation: 0 none, 1 GELU (tanh form)
     float inv_tau[DG_MAX_CANVASES];
 };
+
+// GELU, tanh form (Hendrycks and Gimpel, "Gaussian Error Linear Units", 2016).
+__device__ __forceinline__ float gelu_tanh(float x) {
+    const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
+    return 0.5f * x * (1.0f + tanhf(k0 * fmaf(0.044715f * x, x * x, x)));
+}
+
+// Eight fp32 accumulator values -> eight bf16 (16 bytes), with the epilogue activation.
+__device__ __forceinline__ uint4 pack8_act(const uint32_t* v, int act) {
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = act ? gelu_tanh(__uint_as_float(v[j])) : __uint_as_float(v[j]);
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
 
 template <bool kBf16, int kNT>
 struct Cfg {
@@ -337,15 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         const int row = quarter * 32 + lane;
         const int32_t r = mt * kTileM + row;
         const bool valid = r < p.R;
-        const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
+        const float it = valid && !p.plain ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
-        const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
+        const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
         for (int i = group; i < nkb; i += 2) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             const bool ok = mbar_wait(&lfull[s], ph, wc);
             uint8_t* lt = smem + s * G::kStageBytes + G::kEBytes;
-            if (ok) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
+            if (ok && !p.plain) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
             fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
             if (softmax_group_sync_or(group, !ok)) break;
             if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);
@@ -361,14 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                     if (p.splits == 1) {
                         uint4* dst = reinterpret_cast<uint4*>(p.z + static_cast<size_t>(r) * p.d + col);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            dst[q] = o;
-                        }
+                        for (int q = 0; q < 4; ++q) dst[q] = pack8_act(v + 8 * q, p.act);
                     } else {
                         float4* dst = reinterpret_cast<float4*>(
                             p.partial + (static_cast<size_t>(split) * p.R + r) * p.d + col);
@@ -655,15 +665,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int row = quarter * 32 + lane;
         const int32_t r = mp * 2 * kTileM + static_cast<int>(rank) * kTileM + row;
         const bool valid = r < p.R;
-        const float it = valid ? p.inv_tau[r / p.C] : 1.0f;
+        const float it = valid && !p.plain ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
-        const float nb = valid ? -p.lse[r] * kLog2e : 0.0f;
+        const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
         const int leader_thread = (kFirstSoftmaxWarp + 4 * group) * 32;
         for (int i = group; i < nkb; i += 2) {
             const int s = i % kLS;
             const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, wc);
             uint8_t* lt = lring + s * G::kLStageBytes;
-            if (ok) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
+            if (ok && !p.plain) softmax_row<kBf16>(lt, lt + G::kLBytes, row, a, nb);
             fence_proxy_async_smem();  // each thread's p stores, visible to the tensor core
             if (softmax_group_sync_or(group, !ok)) break;
             if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
@@ -679,14 +689,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     if (p.splits == 1) {
                         uint4* dst = reinterpret_cast<uint4*>(p.z + static_cast<size_t>(r) * p.d + col);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            dst[q] = o;
-                        }
+                        for (int q = 0; q < 4; ++q) dst[q] = pack8_act(v + 8 * q, p.act);
                     } else {
                         float4* dst = reinterpret_cast<float4*>(
                             p.partial + (static_cast<size_t>(split) * p.R + r) * p.d + col);
@@ -729,7 +732,7 @@ __global__ void bounded_wait_test_kernel(long long limit) {
 
 // z[i] = bf16(sum_s partial[s][i]) in a fixed order (deterministic).
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ partial, uint2* __restrict__ z,
-                                                            int64_t n4, int splits) {
+                                                            int64_t n4, int splits, int act) {
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float4 acc = __ldcs(partial + i);
@@ -739,6 +742,12 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
             acc.y += v.y;
             acc.z += v.z;
             acc.w += v.w;
+        }
+        if (act) {
+            acc.x = gelu_tanh(acc.x);
+            acc.y = gelu_tanh(acc.y);
+            acc.z = gelu_tanh(acc.z);
+            acc.w = gelu_tanh(acc.w);
         }
         z[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
@@ -897,6 +906,8 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     kp.total_kb = pl.total_kb;
     kp.wait_limit = sp.wait_limit > 0 ? sp.wait_limit : kWaitLimitCycles;
     kp.fault_block = sp.fault_block;
+    kp.plain = sp.plain_a;
+    kp.act = sp.act;
     std::memcpy(kp.inv_tau, sp.inv_tau, sizeof(kp.inv_tau));
     const int grid = pl.ctas;
 #define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st)
@@ -927,7 +938,7 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     const int64_t n4 = static_cast<int64_t>(sp.R) * sp.d / 4;
     const int blocks = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, 4LL * num_sms()));
     splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(sp.partial),
-                                                reinterpret_cast<uint2*>(sp.z), n4, splits);
+                                                reinterpret_cast<uint2*>(sp.z), n4, splits, sp.act);
     note_launches(1);
     return cudaGetLastError();
 }

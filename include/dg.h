@@ -264,6 +264,25 @@ int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed
                      uint8_t* keep, dg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Feed-forward block on the self-conditioning input (section "Method":     */
+/* z = FFW(p0 E), FFW a standard feed-forward network).  The pages name no  */
+/* architecture; read as a two-layer perceptron without biases,            */
+/*   hidden = gelu(z_in W1),  z_out = hidden W2,                            */
+/* gelu in its tanh form.  Both layers run on the tensor cores (bf16        */
+/* operands, fp32 accumulation); hidden and z_out are stored bf16.          */
+/* z_in: device bf16 [rows, d]; W1: device bf16 [d, d_ff]; W2: device bf16  */
+/* [d_ff, d]; hidden: device bf16 [rows, d_ff] (caller-owned scratch, also  */
+/* an output); z_out: device bf16 [rows, d]; all row-major, 16-byte aligned */
+/* and not aliased.  d, d_ff multiples of 64 in [64, 16384].  Workspace     */
+/* (256-byte aligned, no zeroing needed): dg_ffw_workspace_size bytes (may  */
+/* be 0).  Two contraction launches (+ their split sums) on `stream`.      */
+/* ------------------------------------------------------------------------ */
+size_t dg_ffw_workspace_size(int32_t rows, int32_t d, int32_t d_ff);
+
+int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* W1, const void* W2,
+           void* hidden, void* z_out, void* workspace, size_t workspace_bytes, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Failure-detection test hooks (the pages have no counterpart).  Every wait */
 /* inside the library's kernels is bounded; these entry points make a wait  */
 /* run out on purpose -- without any fault, trap or endless loop -- so that */

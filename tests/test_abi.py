@@ -162,3 +162,15 @@ def test_tau_linear_host_matches_oracle(L):
         assert g == pytest.approx(1.0 / O.tau_linear(t), rel=1e-7)
     out = (ctypes.c_float * 1)()
     assert L.dg_tau_linear((ctypes.c_double * 1)(0.5), 1, ctypes.c_double(0.8), ctypes.c_double(0.0), out) == 1
+
+
+def test_ffw_rejects(L):
+    f = L.dg_ffw
+    ws = L.dg_ffw_workspace_size
+    ws.restype = ctypes.c_size_t
+    assert ws(256, 2048, 8192) > 0 and ws(0, 64, 64) == 0
+    assert f(FAKE, 16, 100, 256, FAKE, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 1 << 30, None) == 1  # d % 64
+    assert f(FAKE, 16, 64, 256, None, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 1 << 30, None) == 1
+    assert f(FAKE, 16, 64, 256, FAKE + 8, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 1 << 30, None) == 2
+    assert f(FAKE, 16, 64, 256, FAKE, FAKE, FAKE, FAKE + 8192, FAKE, 1 << 30, None) == 1  # hidden aliases z_in
+    assert f(FAKE, 256, 2048, 8192, FAKE, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 8, None) == 3  # workspace
