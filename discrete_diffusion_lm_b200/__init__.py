@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.dg_ffw_workspace_size.argtypes = [_i32, _i32, _i32]
         L.dg_ffw_workspace_size.restype = _sz
         L.dg_ffw.argtypes = [_p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _sz, _p]
+        L.dg_sampler_selfcond_step.argtypes = [_p, _int, _i64, _p, _i32, _i32, _i32, _int, _p, _p, _p, _u64, _u32,
+                                               _int, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p, _int, _i32, _p, _p,
+                                               _sz, _p]
         _lib = L
     return _lib
 
@@ -215,6 +218,47 @@ def dg_sampler_step(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V
         _ptr(out.get("lse")), _ptr(out.get("entropy")), _ptr(out.get("branch")),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("dg_sampler_step", rc)
+    return out
+
+
+def dg_sampler_selfcond_step(logits: torch.Tensor, x_t: torch.Tensor, E: torch.Tensor, C: int, t, dt, *,
+                             V: Optional[int] = None, schedule: str = "cosine", inv_tau=None, seed: int = 0,
+                             step: int = 0, mode: str = "sample", out: Optional[dict] = None,
+                             z: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                             ws_z: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """One sampler step and its self-conditioning input z = softmax(L) E in one call (the
+    contraction starts while the logits pass finishes).  Returns the dict of dg_sampler_step's
+    outputs plus "z"."""
+    ld = _row_major_2d(logits, "logits")
+    R = logits.shape[0]
+    V = logits.shape[1] if V is None else V
+    if R % C:
+        raise ValueError("rows must be a multiple of C")
+    B = R // C
+    dev = logits.device
+    d = E.shape[1]
+    if out is None:
+        out = {k: torch.empty(R, dtype=dt_, device=dev) for k, dt_ in
+               (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32),
+                ("max_prob", torch.float32), ("lse", torch.float32), ("entropy", torch.float32),
+                ("branch", torch.uint8))}
+    z = torch.empty((R, d), dtype=torch.bfloat16, device=dev) if z is None else z
+    out["z"] = z
+    if ws is None:
+        ws = workspace("sampler_step", dg_sampler_step_workspace_size(R, V), dev, (R, V), stream)
+    if ws_z is None:
+        nz = dg_selfcond_workspace_size(R, V, d, _dtype_code(logits), _dtype_code(E), True)
+        ws_z = workspace("selfcond", nz, dev, (R, V, d, False, E.dtype), stream)
+    rc = lib().dg_sampler_selfcond_step(
+        _ptr(logits), _dtype_code(logits), ld, _ptr(x_t), B, C, V, DG_SCHED[schedule],
+        _host_doubles(_expand(t, B), B), _host_doubles(_expand(dt, B), B),
+        _host_floats(None if inv_tau is None else _expand(inv_tau, B), B),
+        ctypes.c_uint64(seed), ctypes.c_uint32(step), DG_X0[mode],
+        _ptr(out.get("x_next")), _ptr(out.get("x0_hat")), _ptr(out.get("argmax")), _ptr(out.get("max_prob")),
+        _ptr(out["lse"]), _ptr(out.get("entropy")), _ptr(out.get("branch")),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(E), _dtype_code(E), d, _ptr(z), _ptr(ws_z),
+        ws_z.numel() * ws_z.element_size(), _stream(stream))
+    _check("dg_sampler_selfcond_step", rc)
     return out
 
 

@@ -363,7 +363,7 @@ namespace {
 int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C, int32_t V,
                   const float* inv_tau, const float* lse, const void* E, int embed_dtype, int32_t d, void* z,
                   void* workspace, size_t workspace_bytes, dg_stream_t stream, int32_t fault_block,
-                  long long wait_limit) {
+                  long long wait_limit, bool dependent = false, bool validate_only = false) {
     g_last_error.clear();
     int rc;
     if ((rc = check_logits(logits, logits_dtype, ld, V)) != DG_OK) return rc;
@@ -383,6 +383,7 @@ int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, i
     static thread_local SelfcondParams sp;
     std::memset(&sp, 0, sizeof(sp));
     if ((rc = check_inv_tau(inv_tau, B, sp.inv_tau)) != DG_OK) return rc;
+    if (validate_only) return DG_OK;
     if ((rc = check_device()) != DG_OK) return rc;
 
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -433,6 +434,7 @@ int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, i
     sp.partial = reinterpret_cast<float*>(wp);
     sp.wait_limit = wait_limit;
     sp.fault_block = fault_block;
+    sp.dependent = dependent && lse != nullptr;
     const cudaError_t e = launch_selfcond(sp, s);
     if (e != cudaSuccess) return cuda_fail(e, "self-conditioning launch");
     return DG_OK;
@@ -663,8 +665,8 @@ int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed
 
 size_t dg_ffw_workspace_size(int32_t rows, int32_t d, int32_t d_ff) {
     if (rows < 1 || d < 64 || d_ff < 64) return 0;
-    const size_t a = selfcond_partial_bytes(rows, d, d_ff, true);   // layer 1: K = d, N = d_ff
-    const size_t b = selfcond_partial_bytes(rows, d_ff, d, true);   // layer 2: K = d_ff, N = d
+    const size_t a = selfcond_partial_bytes(rows, d, d_ff, true, true);  // layer 1: K = d, N = d_ff
+    const size_t b = selfcond_partial_bytes(rows, d_ff, d, true, true);  // layer 2: K = d_ff, N = d
     return a > b ? a : b;
 }
 
@@ -709,6 +711,29 @@ int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* 
         if (e != cudaSuccess) return cuda_fail(e, layer == 0 ? "FFW layer 1 launch" : "FFW layer 2 launch");
     }
     return DG_OK;
+}
+
+
+int dg_sampler_selfcond_step(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t, int32_t B,
+                             int32_t C, int32_t V, int schedule, const double* t, const double* dt,
+                             const float* inv_tau, uint64_t seed, uint32_t step, int x0_mode, int32_t* x_next,
+                             int32_t* x0_hat, int32_t* argmax, float* max_prob, float* lse, float* entropy,
+                             uint8_t* branch, void* workspace, size_t workspace_bytes, const void* E,
+                             int embed_dtype, int32_t d, void* z, void* z_workspace, size_t z_workspace_bytes,
+                             dg_stream_t stream) {
+    if (!lse) {
+        g_last_error = "lse is required (the contraction reads it)";
+        return DG_ERR_INVALID_ARG;
+    }
+    // every argument of the contraction is checked before the logits pass is launched
+    int rc = selfcond_impl(logits, logits_dtype, ld, B, C, V, inv_tau, lse, E, embed_dtype, d, z, z_workspace,
+                           z_workspace_bytes, stream, -1, 0, false, true);
+    if (rc != DG_OK) return rc;
+    rc = dg_sampler_step(logits, logits_dtype, ld, x_t, B, C, V, schedule, t, dt, inv_tau, seed, step, x0_mode,
+                         x_next, x0_hat, argmax, max_prob, lse, entropy, branch, workspace, workspace_bytes, stream);
+    if (rc != DG_OK) return rc;
+    return selfcond_impl(logits, logits_dtype, ld, B, C, V, inv_tau, lse, E, embed_dtype, d, z, z_workspace,
+                         z_workspace_bytes, stream, -1, 0, true, false);
 }
 
 }  // extern "C"

@@ -136,6 +136,15 @@ __device__ __forceinline__ void fence_barrier_init() {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while its predecessor in the stream still runs; before it reads anything the
+// predecessor writes it waits for the predecessor's completion (and memory).  A kernel lets its
+// dependents start early by triggering; both are no-ops without such a dependency.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
 // Warp / block reductions (blockDim.x == 32 * kWarpsPerBlock, all threads participate).
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float warp_max(float v) {

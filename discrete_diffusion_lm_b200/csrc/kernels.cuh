@@ -83,10 +83,11 @@ struct SelfcondParams {
     int32_t fault_block;   // test hook: never issue the E copy of this 64-id block (-1: none)
     int32_t plain_a;       // 1: `logits` is a plain bf16 A operand [R, V] (no softmax, lse unused)
     int32_t act;           // epilogue activation on z: 0 none, 1 GELU (tanh form)
+    int32_t dependent;     // 1: launch as a programmatic dependent of the preceding logits pass
     float inv_tau[DG_MAX_CANVASES];
 };
 
-size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16);
+size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16, bool plain_a = false);
 cudaError_t launch_selfcond(const SelfcondParams& p, cudaStream_t s);
 cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t s);
 // One thread waits on a barrier nothing arrives on; the bounded wait must give up (test).

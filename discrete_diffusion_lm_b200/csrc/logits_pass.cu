@@ -423,6 +423,9 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 template <bool kBf16, int kKind>
 __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kernel(const __grid_constant__ PassParams p) {
     __shared__ MergeShared sh;
+    // A contraction launched as a dependent of this pass may start its copies of E and of the logits
+    // (inputs of both) while this pass runs; it waits for the pass to finish before reading lse.
+    if (threadIdx.x == 0) grid_launch_dependents();
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -356,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         const bool valid = r < p.R;
         const float it = valid && !p.plain ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
+        grid_dependency_wait();  // lse comes from the preceding logits pass (a dependent launch)
         const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
         for (int i = group; i < nkb; i += 2) {
             const int s = i % kStages;
@@ -367,7 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
             if (softmax_group_sync_or(group, !ok)) break;
             if (threadIdx.x == 64 + group * kGroupThreads) mbar_arrive(&pready[s]);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, wc))) {
+        const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, wc));
+        grid_launch_dependents();  // the split sum may launch; it waits for this grid's partials
+        if (acc_ok) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
             for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
@@ -451,31 +454,6 @@ __device__ __forceinline__ void cluster_sync() {
 // Arrival on a barrier of another CTA of the cluster (default release semantics).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait with cluster-scope acquire (arrivals may come from the other CTA of the pair).
-__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (aborted(ctl)) return false;
-        if (clock64() - t0 > ctl->limit) {
-            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
-            atomicExch(&g_device_error, 1);
-            return false;
-        }
-    }
 }
 // E box copy whose completion is counted on the pair leader's barrier.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* tm, int32_t c0, int32_t c1,
@@ -667,6 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const bool valid = r < p.R;
         const float it = valid && !p.plain ? p.inv_tau[r / p.C] : 1.0f;
         const float a = it * kLog2e;
+        grid_dependency_wait();  // lse comes from the preceding logits pass (a dependent launch)
         const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
         const int leader_thread = (kFirstSoftmaxWarp + 4 * group) * 32;
         for (int i = group; i < nkb; i += 2) {
@@ -678,7 +657,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (softmax_group_sync_or(group, !ok)) break;
             if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(accum, 0, wc))) {
+        const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, wc));
+        grid_launch_dependents();  // the split sum may launch; it waits for this grid's partials
+        if (acc_ok) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
             for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
@@ -733,6 +714,7 @@ __global__ void bounded_wait_test_kernel(long long limit) {
 // z[i] = bf16(sum_s partial[s][i]) in a fixed order (deterministic).
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ partial, uint2* __restrict__ z,
                                                             int64_t n4, int splits, int act) {
+    grid_dependency_wait();  // launched dependent on the contraction: its partials must be complete
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float4 acc = __ldcs(partial + i);
@@ -812,9 +794,13 @@ struct Plan {
     int ctas;
 };
 
-Plan plan(int R, int V, int d, bool logits_bf16) {
+// Plain-operand GEMMs (the feed-forward block) are short in K: narrow column tiles give enough
+// tiles to fill the GPU without splitting K (and so without a split sum).
+int pick_ntile_plain(int d) { return d % 128 == 0 ? 128 : 64; }
+
+Plan plan(int R, int V, int d, bool logits_bf16, bool plain) {
     Plan pl;
-    const int nt = pick_ntile(d, logits_bf16);
+    const int nt = plain ? pick_ntile_plain(d) : pick_ntile(d, logits_bf16);
     pl.pair = R > kTileM && nt >= 128;
     pl.m_tiles = pl.pair ? (R + 2 * kTileM - 1) / (2 * kTileM) : (R + kTileM - 1) / kTileM;
     pl.n_tiles = d / nt;
@@ -829,8 +815,26 @@ Plan plan(int R, int V, int d, bool logits_bf16) {
     return pl;
 }
 
+// Launch on `st`; with `dependent`, as a programmatic dependent launch of the preceding kernel
+// (it may start early; the kernel waits before reading that kernel's outputs).
+template <typename Kernel, typename Param>
+cudaError_t launch_maybe_dependent(Kernel kernel, int grid, int threads, size_t smem, cudaStream_t st,
+                                   const Param& param, bool dependent) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, param);
+}
+
 template <bool kBf16, int kNT>
-cudaError_t launch_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
+cudaError_t launch_kernel(const KernelParams& kp, int grid, cudaStream_t st, bool dependent) {
     using G = Cfg<kBf16, kNT>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -839,12 +843,11 @@ cudaError_t launch_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
                                         static_cast<int>(G::kSmemBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    selfcond_kernel<kBf16, kNT><<<grid, kThreads, G::kSmemBytes, st>>>(kp);
-    return cudaGetLastError();
+    return launch_maybe_dependent(selfcond_kernel<kBf16, kNT>, grid, kThreads, G::kSmemBytes, st, kp, dependent);
 }
 
 template <bool kBf16, int kNT>
-cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st) {
+cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st, bool dependent) {
     using G = PairCfg<kBf16, kNT>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -853,8 +856,8 @@ cudaError_t launch_pair_kernel(const KernelParams& kp, int grid, cudaStream_t st
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::kSmemBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    selfcond_pair_kernel<kBf16, kNT><<<grid, kPairThreads, G::kSmemBytes, st>>>(kp);
-    return cudaGetLastError();
+    return launch_maybe_dependent(selfcond_pair_kernel<kBf16, kNT>, grid, kPairThreads, G::kSmemBytes, st, kp,
+                                  dependent);
 }
 
 }  // namespace
@@ -871,18 +874,18 @@ int num_sms() {
     return v;
 }
 
-size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16) {
+size_t selfcond_partial_bytes(int32_t R, int32_t V, int32_t d, bool logits_bf16, bool plain) {
     if (R < 1 || V < 1 || d < 64) return 0;
-    const Plan pl = plan(R, V, d, logits_bf16);
+    const Plan pl = plan(R, V, d, logits_bf16, plain);
     return pl.splits > 1 ? static_cast<size_t>(pl.splits) * R * d * sizeof(float) : 0;
 }
 
 cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     static thread_local KernelParams kp;
     std::memset(&kp, 0, sizeof(kp));
-    const Plan pl = plan(sp.R, sp.V, sp.d, sp.logits_bf16 != 0);
+    const Plan pl = plan(sp.R, sp.V, sp.d, sp.logits_bf16 != 0, sp.plain_a != 0);
     const int splits = pl.splits;
-    const int nt = pick_ntile(sp.d, sp.logits_bf16 != 0);
+    const int nt = sp.plain_a ? pick_ntile_plain(sp.d) : pick_ntile(sp.d, sp.logits_bf16 != 0);
     cudaError_t e;
     if (sp.logits_bf16)
         e = encode_2d(&kp.tm_logits, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.logits, sp.V, sp.R,
@@ -910,8 +913,8 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     kp.act = sp.act;
     std::memcpy(kp.inv_tau, sp.inv_tau, sizeof(kp.inv_tau));
     const int grid = pl.ctas;
-#define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st)
-#define DG_PC(BF, NT) e = launch_pair_kernel<BF, NT>(kp, grid, st)
+#define DG_SC(BF, NT) e = launch_kernel<BF, NT>(kp, grid, st, sp.dependent != 0)
+#define DG_PC(BF, NT) e = launch_pair_kernel<BF, NT>(kp, grid, st, sp.dependent != 0)
     if (pl.pair) {
         if (sp.logits_bf16) {
             if (nt == 512) DG_PC(true, 512);
@@ -937,8 +940,19 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     if (e != cudaSuccess || splits == 1) return e;
     const int64_t n4 = static_cast<int64_t>(sp.R) * sp.d / 4;
     const int blocks = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, 4LL * num_sms()));
-    splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(sp.partial),
-                                                reinterpret_cast<uint2*>(sp.z), n4, splits, sp.act);
+    // a dependent launch of the contraction: it may start early and waits for the partials
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, reinterpret_cast<const float4*>(sp.partial),
+                           reinterpret_cast<uint2*>(sp.z), n4, splits, static_cast<int>(sp.act));
+    if (e != cudaSuccess) return e;
     note_launches(1);
     return cudaGetLastError();
 }

@@ -146,6 +146,27 @@ int dg_selfcond(const void* logits, int logits_dtype, int64_t ld, int32_t B, int
                 void* z, void* workspace, size_t workspace_bytes, dg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* One whole sampler step with its self-conditioning input (section         */
+/* "Method": p0, z = p0 E and x_{t-dt} ~ Step(x_t, p0) of one iteration):    */
+/* dg_sampler_step followed by dg_selfcond on the step's own lse, in one    */
+/* call.  The contraction is launched as a programmatic dependent of the    */
+/* logits pass, so its set-up and its copies of E and of the logits overlap */
+/* the end of the pass; it reads lse only after the pass has completed.     */
+/* Arguments: those of dg_sampler_step (lse required), then those of        */
+/* dg_selfcond (E, embed_dtype, d, z and its own workspace, sized by         */
+/* dg_selfcond_workspace_size(B*C, V, d, logits_dtype, embed_dtype, 1)).    */
+/* All arguments are checked before anything is launched.                  */
+/* ------------------------------------------------------------------------ */
+int dg_sampler_selfcond_step(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t,
+                             int32_t B, int32_t C, int32_t V, int schedule, const double* t,
+                             const double* dt, const float* inv_tau, uint64_t seed, uint32_t step,
+                             int x0_mode, int32_t* x_next, int32_t* x0_hat, int32_t* argmax,
+                             float* max_prob, float* lse, float* entropy, uint8_t* branch,
+                             void* workspace, size_t workspace_bytes, const void* E,
+                             int embed_dtype, int32_t d, void* z, void* z_workspace,
+                             size_t z_workspace_bytes, dg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Training-side forward corruption (section "Method": forward path, noisy   */
 /* tokens drawn uniformly from the vocabulary; section "Dataset": P + K*C    */
 /* layout, one loss canvas per sequence chosen uniformly).                   */

@@ -131,3 +131,24 @@ def test_one_hot_rows_pick_embedding_rows():
     z = dg_selfcond(logits.to(torch.bfloat16), E, R)
     torch.cuda.synchronize()
     torch.testing.assert_close(z.float(), E[ids].float(), atol=1e-2, rtol=1e-2)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid", "full"])
+def test_fused_step_equals_separate_calls(name):
+    # the fused entry point launches the contraction as a dependent of the logits pass; its
+    # results must equal the two separate calls exactly (same kernels, same order of sums)
+    cfg = W.SAMPLER_CONFIGS[name]
+    logits = W.make_logits(cfg, DEV)
+    E = W.make_embedding(cfg, DEV)
+    x_t = W.make_canvas(cfg, DEV)
+    t, dt = cfg.times(1)
+    sep = dg.dg_sampler_step(logits, x_t, cfg.C, t, dt, schedule=cfg.schedule, seed=4, step=1)
+    z_sep = dg.dg_selfcond(logits, E, cfg.C, lse=sep["lse"])
+    torch.cuda.synchronize()
+    for _ in range(3):  # repeated: any early read of lse would show as a difference
+        fused = dg.dg_sampler_selfcond_step(logits, x_t, E, cfg.C, t, dt, schedule=cfg.schedule, seed=4, step=1)
+        torch.cuda.synchronize()
+        for k in ("x_next", "x0_hat", "argmax", "max_prob", "lse", "entropy", "branch"):
+            assert torch.equal(fused[k], sep[k]), k
+        assert torch.equal(fused["z"], z_sep)
+    assert dg.dg_device_error() == 0
