@@ -112,9 +112,9 @@ int32_t n_chunks_of(int32_t V) { return (V + kChunk - 1) / kChunk; }
 int32_t n_groups_of(int32_t V) { return (V + 4 * kChunk - 1) / (4 * kChunk); }
 int32_t groups_per_cta_of(int32_t /*n_groups*/) { return kPassWarps; }
 
-// Logits-pass workspace: row tickets, sequence tickets, then the chunk records.
+// Logits-pass workspace: per-row counters, sequence tickets (canvas CE), then the chunk records.
 struct PassWs {
-    uint32_t* row_ticket;
+    unsigned* row_count;
     uint32_t* seq_ticket;
     float4* rec;
 };
@@ -125,7 +125,7 @@ size_t pass_ws_bytes(int32_t R, int32_t V, int32_t n_seq) {
 PassWs carve_pass_ws(void* ws, int32_t R, int32_t n_seq) {
     char* p = static_cast<char*>(ws);
     PassWs w;
-    w.row_ticket = reinterpret_cast<uint32_t*>(p);
+    w.row_count = reinterpret_cast<unsigned*>(p);
     p += align_up(static_cast<size_t>(R) * 4, 256);
     w.seq_ticket = reinterpret_cast<uint32_t*>(p);
     p += align_up(static_cast<size_t>(n_seq) * 4, 256);
@@ -190,8 +190,11 @@ int dg_device_error(int* code) {
     if ((rc = check_device()) != DG_OK) return rc;
     const cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    const cudaError_t r = read_and_clear_device_error(code);
-    if (r != cudaSuccess) return cuda_fail(r, "reading the device error word");
+    int c1 = 0, c2 = 0;
+    cudaError_t r = read_and_clear_device_error(&c1);
+    if (r == cudaSuccess) r = read_and_clear_pass_error(&c2);
+    if (r != cudaSuccess) return cuda_fail(r, "reading the device error words");
+    *code = c1 ? c1 : c2;
     return DG_OK;
 }
 
@@ -242,7 +245,7 @@ int dg_sampler_step(const void* logits, int logits_dtype, int64_t ld, const int3
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_ticket = w.row_ticket;
+    p.row_count = w.row_count;
     p.x_t = x_t;
     p.key0 = static_cast<uint32_t>(seed);
     p.key1 = static_cast<uint32_t>(seed >> 32);
@@ -331,7 +334,7 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_ticket = w.row_ticket;
+    p.row_count = w.row_count;
     p.seq_ticket = w.seq_ticket;
     p.x0 = x0;
     p.canvas_idx = canvas_idx;
@@ -405,7 +408,7 @@ int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, i
         p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
         p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
         p.rec = w.rec;
-        p.row_ticket = w.row_ticket;
+        p.row_count = w.row_count;
         p.lse = lse_ws;
         std::memcpy(p.inv_tau, sp.inv_tau, sizeof(float) * B);
         const cudaError_t e = launch_logits_pass(p, kPassStats, logits_dtype == DG_BF16, s);
@@ -576,7 +579,7 @@ int dg_sampler_step_eb(const void* logits, int logits_dtype, int64_t ld, int32_t
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_ticket = w.row_ticket;
+    p.row_count = w.row_count;
     p.key0 = static_cast<uint32_t>(seed);
     p.key1 = static_cast<uint32_t>(seed >> 32);
     p.step = step;

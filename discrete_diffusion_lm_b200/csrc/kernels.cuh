@@ -25,7 +25,7 @@ struct PassParams {
     int32_t groups_per_cta;  // 4-chunk groups per CTA, a multiple of the warps per CTA
     int32_t segs;            // CTAs per row
     float4* rec;             // [R, n_chunks] per-chunk (raw max, S, T, -)
-    uint32_t* row_ticket;    // [R], zero between calls
+    unsigned* row_count;     // [R] streaming CTAs done per row; zero between calls
     // sampler
     const int32_t* x_t;
     uint32_t key0, key1, step;
@@ -56,6 +56,8 @@ constexpr int kPassThreads = 128;
 constexpr int kPassWarps = kPassThreads / 32;
 
 cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s);
+// Reads and clears the logits pass's device error word (1 = a merge's bounded wait expired).
+cudaError_t read_and_clear_pass_error(int* out);
 
 struct NoiseParams {
     const int32_t* x0;

@@ -11,16 +11,32 @@
 //   warp-load); each 8-lane subgroup computes its chunk's raw maximum, S = sum exp(l' - m') and
 //   T = sum exp(l' - m')(l' - m') with l' = l * inv_tau and m' = max l', and writes one 16-byte
 //   record per chunk.
-// Phase 2 (the last CTA to finish a row, found by an atomic ticket -- nobody waits): merges the
-//   row's chunk records into lse, max-prob and entropy, finds the argmax, draws x0_hat by two-level
+// Phase 2 (merge_kernel, one CTA per row, launched as a programmatic dependent of phase 1 once every
+//   phase-1 CTA has started; each merge waits only for its own row, whose streaming CTAs count
+//   their records with a release increment and do not wait themselves): merges the row's chunk
+//   records into lse, max-prob and entropy, finds the argmax, draws x0_hat by two-level
 //   Gumbel-max (level 1 over chunk records, level 2 by re-reading the winning chunk from L2), and
-//   samples the Step posterior with one Philox draw.  It leaves the ticket at zero.
+//   samples the Step posterior with one Philox draw.  Rows finish streaming in order, so most
+//   merges run while later rows still stream.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace dg {
 
 namespace {
+
+// Device error word of the logits pass: set when a merge's bounded wait expires.
+__device__ int g_pass_error = 0;
+constexpr long long kMergeWaitLimit = 4000000000LL;  // SM cycles, about 2 s
+
+__device__ __forceinline__ void red_release_add(unsigned* addr, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* addr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
+}
 
 // bf16 -1.0e30 (0xF14A), used twice in a 32-bit word: -inf logits are clamped to it so that the
 // entropy sum never forms 0 * -inf.
@@ -163,13 +179,62 @@ __device__ __noinline__ ChunkStats group_ragged(const void* row, bool bf16, int3
     return finish(m_raw, s, t, nbig);
 }
 
+// Four consecutive logits [v, v + 4) of a row as raw words (bf16: 8 bytes, fp32: 16 bytes); one
+// vector load when the quad lies inside [.., hi), element loads at the ragged end.
+struct RawQuad {
+    uint32_t w[4];
+};
+template <bool kBf16>
+__device__ __forceinline__ RawQuad load_quad(const void* row, int32_t v, int32_t hi) {
+    RawQuad q;
+    if (v + 4 <= hi) {
+        if (kBf16) {
+            const uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(row) + v);
+            q.w[0] = x.x;
+            q.w[1] = x.y;
+            q.w[2] = q.w[3] = 0u;
+        } else {
+            const uint4 x = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(row) + v);
+            q.w[0] = x.x;
+            q.w[1] = x.y;
+            q.w[2] = x.z;
+            q.w[3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q.w[k] = v + k < hi ? __float_as_uint(load_logit(row, v + k, kBf16)) : 0u;
+    }
+    return q;
+}
+// The quad as clamped floats; ids at or past hi are -inf.
+template <bool kBf16>
+__device__ __forceinline__ void unpack_quad(const RawQuad& q, int32_t v, int32_t hi, float nbig, float (&out)[4]) {
+    if (v + 4 <= hi && kBf16) {
+        out[0] = bf16_lo(q.w[0]);
+        out[1] = bf16_hi(q.w[0]);
+        out[2] = bf16_lo(q.w[1]);
+        out[3] = bf16_hi(q.w[1]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) out[k] = __uint_as_float(q.w[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[k] = v + k < hi ? fmaxf(out[k], nbig) : -INFINITY;
+}
+
+// Level-1 Gumbel score of a chunk: its log-sum-exp of l' plus a Gumbel variate (-inf for a chunk
+// without mass).
+__device__ __forceinline__ float chunk_score(float m_raw, float S, float inv_tau, uint32_t word) {
+    return (m_raw * inv_tau + logf(S)) + gumbel_from_word(word);
+}
+
 struct MergeShared {
     float f[2 * kPassWarps];
     int i[2 * kPassWarps];
     int flag;
 };
 
-// Per-row merge, run by the last CTA of the row.  Global memory is visited in two round trips:
+// Per-row merge, run by the merge kernel's CTA of the row.  Global memory is visited in two round trips:
 // the chunk records (thread t holds quads of four consecutive chunks 4q .. 4q+3, q = t + u T, in
 // registers, so one Philox call serves four chunk Gumbel variates), then the two chunks that must
 // be re-read (the one holding the argmax and the level-1 winner), fetched together.
@@ -190,9 +255,6 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const float4* rec = p.rec + static_cast<size_t>(row) * nch;
     const float nbig = neg_big(kBf16);
 
-    // Scalars needed at the very end, loaded first so their latency overlaps the merge.
-    int32_t xt = 0;
-    if (kKind == kPassSampler && tid == 0 && p.x_t) xt = p.x_t[row];
     float target_logit = 0.f;
     bool target_ok = false;
     int32_t b_seq = 0, i_seq = 0;
@@ -219,6 +281,20 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             const int32_t j = 4 * (tid + u * kPassThreads) + k;
             r[u][k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
         }
+    // What thread 0 needs at the very end, fetched or computed while the records are in flight:
+    // the current token, the canvas's Step thresholds and the Step's Philox words.
+    int32_t xt = 0;
+    unsigned long long thr_sd = 0, thr_jd = 0, thr_ss = 0;
+    uint4 step_w = make_uint4(0u, 0u, 0u, 0u);
+    if (kKind == kPassSampler && tid == 0 && p.x_next) {
+        xt = p.x_t[row];
+        thr_sd = p.thr_stay_diff[canvas];
+        thr_jd = p.thr_jump_diff[canvas];
+        thr_ss = p.thr_stay_same[canvas];
+        step_w = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), p.step, kDomStep), p.key0, p.key1);
+        // pin the words here: computed while the records are in flight, not at the end
+        asm volatile("" ::"r"(step_w.x), "r"(step_w.y), "l"(thr_sd), "l"(thr_jd), "l"(thr_ss), "r"(xt));
+    }
     // Records beyond those (rows longer than 262144 ids) are re-read from L2 in each pass.
     constexpr int kFar = kRecQuads * kPassThreads;
     auto far_quad = [&](int32_t q, float4 (&f)[4]) {
@@ -249,7 +325,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             for (int k = 0; k < 4; ++k) {
                 const int32_t j = 4 * q + k;
                 if (j < nch) {
-                    const float sc = (f[k].x * inv_tau + logf(f[k].y)) + gumbel_from_word(word_of(w, k));
+                    const float sc = chunk_score(f[k].x, f[k].y, inv_tau, word_of(w, k));
                     if (sc > bs) {
                         bs = sc;
                         bj = j;
@@ -272,19 +348,18 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     if (!sampling || bj >= nch) bj = jm;  // greedy, or NaN scores only
     const float m_row = m_raw * inv_tau;
 
-    // Both re-read chunks are known: ids lo + 4 tid .. lo + 4 tid + 3 of each, loaded now.
-    float av[kQuads][4], gv[kQuads][4];
+    // Both re-read chunks are known: quads of ids lo + 4 (tid + u T) .. + 3 of each, loaded now as
+    // raw words and used only after the next exchange, so the loads overlap it.
     const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
     const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
+    RawQuad araw[kQuads], graw[kQuads];
     if (kKind == kPassSampler) {
 #pragma unroll
-        for (int u = 0; u < kQuads; ++u)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int32_t o = 4 * (tid + u * kPassThreads) + k;
-                av[u][k] = alo + o < ahi ? fmaxf(load_logit(rowp, alo + o, kBf16), nbig) : -INFINITY;
-                gv[u][k] = glo + o < ghi ? fmaxf(load_logit(rowp, glo + o, kBf16), nbig) : -INFINITY;
-            }
+        for (int u = 0; u < kQuads; ++u) {
+            const int32_t o = 4 * (tid + u * kPassThreads);
+            araw[u] = load_quad<kBf16>(rowp, alo + o, ahi);
+            graw[u] = load_quad<kBf16>(rowp, glo + o, ghi);
+        }
     }
 
     // (2) Log-sum-exp merge of (S, T) relative to the row maximum.
@@ -314,7 +389,6 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     if (kKind == kPassStats) {
         if (tid == 0) {
             p.lse[row] = lse;
-            p.row_ticket[row] = 0u;
         }
         return;
     }
@@ -324,7 +398,6 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             const float loss = target_ok ? lse - target_logit : __int_as_float(0x7fc00000);  // NaN: bad target
             p.loss_rows[row] = loss;
             if (p.lse) p.lse[row] = lse;
-            p.row_ticket[row] = 0u;
             __threadfence();
             const unsigned prev = atomicAdd(&p.seq_ticket[b_seq], 1u);
             const bool last = prev == static_cast<unsigned>(p.C - 1);
@@ -348,6 +421,13 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     // ---- sampler epilogue
     // (3) The first id of the argmax chunk holding the row maximum, and the level-2 winner
     // argmax of l'_v + G_v over the level-1 chunk (four ids per Philox call).
+    float av[kQuads][4], gv[kQuads][4];
+#pragma unroll
+    for (int u = 0; u < kQuads; ++u) {
+        const int32_t o = 4 * (tid + u * kPassThreads);
+        unpack_quad<kBf16>(araw[u], alo + o, ahi, nbig, av[u]);
+        unpack_quad<kBf16>(graw[u], glo + o, ghi, nbig, gv[u]);
+    }
     float amv = -INFINITY;
     int am = 0x7fffffff;
 #pragma unroll
@@ -387,14 +467,13 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         if (p.x_next) {  // the Step posterior (skipped when a per-canvas rule decides instead)
             unsigned long long t_stay, t_jump;
             if (x0 != xt) {
-                t_stay = p.thr_stay_diff[canvas];
-                t_jump = p.thr_jump_diff[canvas];
+                t_stay = thr_sd;
+                t_jump = thr_jd;
             } else {
-                t_stay = p.thr_stay_same[canvas];
+                t_stay = thr_ss;
                 t_jump = t_stay;
             }
-            const uint4 w =
-                philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), p.step, kDomStep), p.key0, p.key1);
+            const uint4 w = step_w;
             const unsigned long long u = w.x;
             int32_t xn;
             uint8_t br;
@@ -416,15 +495,13 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         if (p.max_prob) p.max_prob[row] = 1.0f / S;
         if (p.lse) p.lse[row] = lse;
         if (p.entropy) p.entropy[row] = ln_s - T / S;
-        p.row_ticket[row] = 0u;
     }
 }
 
 template <bool kBf16, int kKind>
 __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kernel(const __grid_constant__ PassParams p) {
-    __shared__ MergeShared sh;
-    // A contraction launched as a dependent of this pass may start its copies of E and of the logits
-    // (inputs of both) while this pass runs; it waits for the pass to finish before reading lse.
+    // The merge kernel, launched as a programmatic dependent, may start once every CTA of this grid
+    // has started; it waits for this grid to finish before reading the chunk records.
     if (threadIdx.x == 0) grid_launch_dependents();
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;
@@ -450,19 +527,41 @@ __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kern
         const int32_t c = 4 * gi + (lane >> 3);
         if ((lane & 7) == 0 && c < p.n_chunks) rec[c] = make_float4(cs.m_raw, cs.S, cs.T, 0.f);
     }
-    // The barrier orders every warp's record stores before thread 0's fence, and the fence is
-    // cumulative: one fence makes the whole CTA's records visible before its ticket increment.
-    // The last CTA of the row fences once more (acquire) before its threads read the records.
+    // Count this CTA's records for the row: the barrier orders every warp's record stores before
+    // thread 0's release increment (fire-and-forget), which the row's merge acquires.
     __syncthreads();
+    if (threadIdx.x == 0) red_release_add(&p.row_count[row], 1u);
+}
+
+// Per-row merge of the chunk records: one CTA per row, launched as a programmatic dependent of the
+// streaming kernel.  Its own dependents (a contraction reading lse) may start as soon as every
+// merge CTA has started; they wait for the merges to finish.
+template <bool kBf16, int kKind>
+__global__ void __launch_bounds__(kPassThreads) merge_kernel(const __grid_constant__ PassParams p) {
+    __shared__ MergeShared sh;
+    if (threadIdx.x == 0) grid_launch_dependents();
+    const int32_t row = blockIdx.x;
+    // Wait (bounded) until all p.segs CTAs of the row have counted their records.  Every streaming
+    // CTA has started before this grid launches, so the wait depends on no CTA still to be placed.
     if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(&p.row_ticket[row], 1u);
-        const bool last = prev == static_cast<unsigned>(p.segs - 1);
-        if (last) __threadfence();
-        sh.flag = last;
+        const unsigned target = static_cast<unsigned>(p.segs);
+        if (ld_acquire(&p.row_count[row]) < target) {
+            const long long t0 = clock64();
+            while (ld_acquire(&p.row_count[row]) < target) {
+                __nanosleep(256);
+                if (clock64() - t0 > kMergeWaitLimit) {
+                    atomicExch(&g_pass_error, 1);
+                    break;
+                }
+            }
+        }
+        p.row_count[row] = 0u;  // ready for the next call (its streaming kernel starts after this grid ends)
     }
     __syncthreads();
-    if (!sh.flag) return;
+    const int32_t canvas = row / p.C;
+    const float inv_tau = kKind == kPassCE ? 1.0f : p.inv_tau[canvas];
+    constexpr int kElt = kBf16 ? 2 : 4;
+    const char* rowp = reinterpret_cast<const char*>(p.logits) + static_cast<size_t>(row) * p.ld * kElt;
     merge_row<kBf16, kKind>(p, row, canvas, inv_tau, rowp, sh);
 }
 
@@ -471,8 +570,25 @@ __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kern
 cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s) {
     const long long grid = static_cast<long long>(p.R) * p.segs;
     if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (p.groups_per_cta != kPassWarps) return cudaErrorInvalidValue;  // the kernel maps one group per warp
     const dim3 g(static_cast<unsigned>(grid)), b(kPassThreads);
-#define DG_LAUNCH(BF, K) logits_pass_kernel<BF, K><<<g, b, 0, s>>>(p)
+    // the merge: one CTA per row, a programmatic dependent of the streaming kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.R));
+    cfg.blockDim = b;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaSuccess;
+#define DG_LAUNCH(BF, K)                                                  \
+    do {                                                                  \
+        logits_pass_kernel<BF, K><<<g, b, 0, s>>>(p);                     \
+        e = cudaGetLastError();                                           \
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, merge_kernel<BF, K>, p); \
+    } while (0)
     if (is_bf16) {
         if (kind == kPassSampler) DG_LAUNCH(true, kPassSampler);
         else if (kind == kPassStats) DG_LAUNCH(true, kPassStats);
@@ -483,8 +599,20 @@ cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaS
         else DG_LAUNCH(false, kPassCE);
     }
 #undef DG_LAUNCH
-    note_launches(1);
-    return cudaGetLastError();
+    note_launches(2);
+    return e;
+}
+
+cudaError_t read_and_clear_pass_error(int* out) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_pass_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_pass_error, &zero, sizeof(int));
+    }
+    *out = v;
+    return e;
 }
 
 }  // namespace dg
