@@ -279,6 +279,7 @@ def run_ours(args, rank, world, local):
     train = bench_train(dg, W, dev, stream, hbm)
     eb = bench_eb(dg, W, dev, stream, bufs, hbm)
     ffw = bench_ffw(dg, W, dev, stream, peaks)
+    configs = bench_configs(dg, W, dev, stream, peaks)
 
     # ---- end to end through the public API with host buffers
     e2e = bench_e2e(dg, W, cfg, dev, E, args, world, barrier)
@@ -313,6 +314,7 @@ def run_ours(args, rank, world, local):
             "train": train,
             "entropy_bounded": eb,
             "ffw": ffw,
+            "other_workloads": configs,
         },
         "e2e": e2e,
         "gpu_launches": int(round(launches_per_step * K)),
@@ -432,6 +434,57 @@ def bench_ffw(dg, W, dev, stream, peaks):
                         "(L2-resident across replays)",
             "ffw_us": round(us, 2), "ffw_TFLOPs": round(flops / (us * 1e-6) / 1e12, 1),
             "ffw_frac_of_slower_bound": round(bound_us / us, 4), "slower_bound_us": round(bound_us, 2)}
+
+
+def bench_configs(dg, W, dev, stream, peaks):
+    """Per-kernel times of the other sampler workloads (logits pass incl. merge; contraction incl.
+    split sum), graph replays after warm-up; tiny and mid fit in L2 (times only)."""
+    import torch
+    hbm = peaks["hbm_gbs"]
+    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    out = {}
+    for name in ("tiny", "mid", "batched"):
+        cfg = W.SAMPLER_CONFIGS[name]
+        logits = W.make_logits(cfg, dev)
+        E = W.make_embedding(cfg, dev)
+        x_t = W.make_canvas(cfg, dev)
+        t, dt = cfg.times(1)
+        o = dg.dg_sampler_step(logits, x_t, cfg.C, t, dt, schedule=cfg.schedule, stream=stream)
+        z = dg.dg_selfcond(logits, E, cfg.C, lse=o["lse"], stream=stream)
+        stream.synchronize()
+        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            dg.dg_sampler_step(logits, x_t, cfg.C, t, dt, schedule=cfg.schedule, out=o, stream=stream)
+        with torch.cuda.graph(g2, stream=stream):
+            dg.dg_selfcond(logits, E, cfg.C, lse=o["lse"], z=z, stream=stream)
+        reps = 10
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g1.replay()
+                g2.replay()
+            e[0].record(stream)
+            for _ in range(reps):
+                g1.replay()
+            e[1].record(stream)
+            for _ in range(reps):
+                g2.replay()
+            e[2].record(stream)
+        stream.synchronize()
+        k1 = e[0].elapsed_time(e[1]) * 1e3 / reps
+        k2 = e[1].elapsed_time(e[2]) * 1e3 / reps
+        lbytes = logits.numel() * logits.element_size()
+        flops = 2.0 * cfg.R * cfg.V * cfg.d
+        out[name] = {"R": cfg.R, "V": cfg.V, "d": cfg.d, "logits_pass_us": round(k1, 2), "selfcond_us": round(k2, 2),
+                     "step_us": round(k1 + k2, 2), "selfcond_TFLOPs": round(flops / (k2 * 1e-6) / 1e12, 1)}
+        if name == "batched":
+            out[name]["logits_pass_frac_hbm"] = round(lbytes / (k1 * 1e-6) / 1e9 / hbm, 4)
+            out[name]["selfcond_frac_tensor_sustained"] = round(flops / (k2 * 1e-6) / 1e12 / tc, 4)
+        else:
+            out[name]["note"] = "inputs fit in L2: times only"
+        del logits, E, x_t, o, z, g1, g2
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_eb(dg, W, dev, stream, bufs, hbm):

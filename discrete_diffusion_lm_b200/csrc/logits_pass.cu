@@ -222,10 +222,10 @@ __device__ __forceinline__ void unpack_quad(const RawQuad& q, int32_t v, int32_t
     for (int k = 0; k < 4; ++k) out[k] = v + k < hi ? fmaxf(out[k], nbig) : -INFINITY;
 }
 
-// Level-1 Gumbel score of a chunk: its log-sum-exp of l' plus a Gumbel variate (-inf for a chunk
+// Level-1 Gumbel score of a chunk: its log-sum-exp of l' plus its Gumbel variate (-inf for a chunk
 // without mass).
-__device__ __forceinline__ float chunk_score(float m_raw, float S, float inv_tau, uint32_t word) {
-    return (m_raw * inv_tau + logf(S)) + gumbel_from_word(word);
+__device__ __forceinline__ float chunk_score(float m_raw, float S, float inv_tau, float gumbel) {
+    return (m_raw * inv_tau + logf(S)) + gumbel;
 }
 
 struct MergeShared {
@@ -254,6 +254,45 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     const int32_t nch = p.n_chunks;
     const float4* rec = p.rec + static_cast<size_t>(row) * nch;
     const float nbig = neg_big(kBf16);
+    const bool sampling = kKind == kPassSampler && p.mode != DG_X0_GREEDY;
+
+    // The chunk Gumbel variates depend only on (seed, step, row, chunk): computed before the row's
+    // records are ready, while its last streaming CTAs may still run.
+    float gum[kRecQuads][4];
+#pragma unroll
+    for (int u = 0; u < kRecQuads; ++u) {
+        const int32_t q = tid + u * kPassThreads;
+        if (sampling && 4 * q < nch) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
+                p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) gum[u][k] = gumbel_from_word(word_of(w, k));
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) gum[u][k] = 0.f;
+        }
+        // pin: computed here, before the wait, not where the scores are formed
+        asm volatile("" ::"f"(gum[u][0]), "f"(gum[u][1]), "f"(gum[u][2]), "f"(gum[u][3]));
+    }
+    // Wait (bounded) until all p.segs streaming CTAs of the row have counted their records.  Every
+    // streaming CTA has started before this grid launches, so the wait depends on no CTA still to
+    // be placed.
+    if (tid == 0) {
+        const unsigned target = static_cast<unsigned>(p.segs);
+        if (ld_acquire(&p.row_count[row]) < target) {
+            const long long t0 = clock64();
+            while (ld_acquire(&p.row_count[row]) < target) {
+                __nanosleep(128);
+                if (clock64() - t0 > kMergeWaitLimit) {
+                    atomicExch(&g_pass_error, 1);
+                    break;
+                }
+            }
+        }
+        p.row_count[row] = 0u;  // ready for the next call (its streaming kernel starts after this grid ends)
+    }
+    __syncthreads();
 
     float target_logit = 0.f;
     bool target_ok = false;
@@ -306,11 +345,10 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     };
 
     // (1) The first chunk holding the row maximum of the raw chunk maxima, and the level-1 winner
-    // of the chunk scores lse_c + G_c (four chunks per Philox call).
-    const bool sampling = kKind == kPassSampler && p.mode != DG_X0_GREEDY;
+    // of the chunk scores lse_c + G_c.
     float mv = -INFINITY, bs = -INFINITY;
     int jm = 0x7fffffff, bj = 0x7fffffff;
-    auto scan_quad = [&](int32_t q, const float4 (&f)[4]) {
+    auto scan_quad = [&](int32_t q, const float4 (&f)[4], const float (&g)[4]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             if (f[k].x > mv) {  // ascending ids, strict: the first maximum wins
@@ -318,14 +356,11 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
                 jm = 4 * q + k;
             }
         if (sampling) {
-            const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
-                p.key1);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int32_t j = 4 * q + k;
                 if (j < nch) {
-                    const float sc = chunk_score(f[k].x, f[k].y, inv_tau, word_of(w, k));
+                    const float sc = chunk_score(f[k].x, f[k].y, inv_tau, g[k]);
                     if (sc > bs) {
                         bs = sc;
                         bj = j;
@@ -336,11 +371,19 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     };
 #pragma unroll
     for (int u = 0; u < kRecQuads; ++u)
-        if (4 * (tid + u * kPassThreads) < nch) scan_quad(tid + u * kPassThreads, r[u]);
+        if (4 * (tid + u * kPassThreads) < nch) scan_quad(tid + u * kPassThreads, r[u], gum[u]);
     for (int32_t q = tid + kFar; 4 * q < nch; q += kPassThreads) {
         float4 f[4];
         far_quad(q, f);
-        scan_quad(q, f);
+        float g[4] = {0.f, 0.f, 0.f, 0.f};
+        if (sampling) {
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(row), p.step, kDomChunkGumbel), p.key0,
+                p.key1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) g[k] = gumbel_from_word(word_of(w, k));
+        }
+        scan_quad(q, f, g);
     }
     block_argmax2<kPassWarps>(mv, jm, bs, bj, sh.f, sh.i);
     const float m_raw = mv;
@@ -541,23 +584,6 @@ __global__ void __launch_bounds__(kPassThreads) merge_kernel(const __grid_consta
     __shared__ MergeShared sh;
     if (threadIdx.x == 0) grid_launch_dependents();
     const int32_t row = blockIdx.x;
-    // Wait (bounded) until all p.segs CTAs of the row have counted their records.  Every streaming
-    // CTA has started before this grid launches, so the wait depends on no CTA still to be placed.
-    if (threadIdx.x == 0) {
-        const unsigned target = static_cast<unsigned>(p.segs);
-        if (ld_acquire(&p.row_count[row]) < target) {
-            const long long t0 = clock64();
-            while (ld_acquire(&p.row_count[row]) < target) {
-                __nanosleep(256);
-                if (clock64() - t0 > kMergeWaitLimit) {
-                    atomicExch(&g_pass_error, 1);
-                    break;
-                }
-            }
-        }
-        p.row_count[row] = 0u;  // ready for the next call (its streaming kernel starts after this grid ends)
-    }
-    __syncthreads();
     const int32_t canvas = row / p.C;
     const float inv_tau = kKind == kPassCE ? 1.0f : p.inv_tau[canvas];
     constexpr int kElt = kBf16 ? 2 : 4;
