@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
         L.dg_launch_count.restype = _u64
         L.dg_device_error.argtypes = [_p]
         L.dg_test_bounded_wait.argtypes = [_u32, _p]
+        L.dg_test_merge_stall.argtypes = [_p, _int, _i64, _i32, _i32, _p, _p, _sz, _u32, _p]
         L.dg_test_selfcond_stall.argtypes = [_p, _int, _i64, _i32, _i32, _i32, _p, _p, _p, _int, _i32, _p, _p, _sz,
                                              _p, _i32, _u32]
         L.dg_sampler_step_workspace_size.argtypes = [_i32, _i32]

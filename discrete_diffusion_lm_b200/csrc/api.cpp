@@ -739,4 +739,37 @@ int dg_sampler_selfcond_step(const void* logits, int logits_dtype, int64_t ld, c
                          z_workspace_bytes, stream, -1, 0, true, false);
 }
 
+
+int dg_test_merge_stall(const void* logits, int logits_dtype, int64_t ld, int32_t rows, int32_t V, float* lse,
+                        void* workspace, size_t workspace_bytes, uint32_t limit_cycles, dg_stream_t stream) {
+    g_last_error.clear();
+    int rc;
+    if ((rc = check_logits(logits, logits_dtype, ld, V)) != DG_OK) return rc;
+    if (rows < 1 || !lse) return fail(DG_ERR_INVALID_ARG, "rows >= 1 and lse are required");
+    if (limit_cycles == 0) return fail(DG_ERR_INVALID_ARG, "limit_cycles must be > 0");
+    const size_t need = pass_ws_bytes(rows, V, 0);
+    if (!workspace || workspace_bytes < need)
+        return fail(DG_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+    if ((rc = check_device()) != DG_OK) return rc;
+    static thread_local PassParams p;
+    std::memset(&p, 0, sizeof(p));
+    const PassWs w = carve_pass_ws(workspace, rows, 0);
+    p.logits = logits;
+    p.ld = ld;
+    p.R = rows;
+    p.C = rows;
+    p.V = V;
+    p.n_chunks = n_chunks_of(V);
+    p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
+    p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
+    p.rec = w.rec;
+    p.row_count = w.row_count;
+    p.lse = lse;
+    p.inv_tau[0] = 1.0f;
+    p.merge_wait_limit = static_cast<long long>(limit_cycles);
+    const cudaError_t e = launch_merge_only(p, logits_dtype == DG_BF16, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "merge stall test launch");
+    return DG_OK;
+}
+
 }  // extern "C"

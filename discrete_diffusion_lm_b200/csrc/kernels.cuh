@@ -26,6 +26,7 @@ struct PassParams {
     int32_t segs;            // CTAs per row
     float4* rec;             // [R, n_chunks] per-chunk (raw max, S, T, -)
     unsigned* row_count;     // [R] streaming CTAs done per row; zero between calls
+    long long merge_wait_limit;  // cycles a merge waits for its row (0: the library default)
     // sampler
     const int32_t* x_t;
     uint32_t key0, key1, step;
@@ -56,6 +57,8 @@ constexpr int kPassThreads = 128;
 constexpr int kPassWarps = kPassThreads / 32;
 
 cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s);
+// Test hook: the statistics merge kernel alone, with nothing counting the rows (its waits expire).
+cudaError_t launch_merge_only(const PassParams& p, int is_bf16, cudaStream_t s);
 // Reads and clears the logits pass's device error word (1 = a merge's bounded wait expired).
 cudaError_t read_and_clear_pass_error(int* out);
 

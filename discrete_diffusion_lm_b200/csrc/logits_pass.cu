@@ -282,9 +282,10 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         const unsigned target = static_cast<unsigned>(p.segs);
         if (ld_acquire(&p.row_count[row]) < target) {
             const long long t0 = clock64();
+            const long long limit = p.merge_wait_limit > 0 ? p.merge_wait_limit : kMergeWaitLimit;
             while (ld_acquire(&p.row_count[row]) < target) {
                 __nanosleep(128);
-                if (clock64() - t0 > kMergeWaitLimit) {
+                if (clock64() - t0 > limit) {
                     atomicExch(&g_pass_error, 1);
                     break;
                 }
@@ -627,6 +628,14 @@ cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaS
 #undef DG_LAUNCH
     note_launches(2);
     return e;
+}
+
+cudaError_t launch_merge_only(const PassParams& p, int is_bf16, cudaStream_t s) {
+    if (p.R < 1) return cudaErrorInvalidConfiguration;
+    if (is_bf16) merge_kernel<true, kPassStats><<<p.R, kPassThreads, 0, s>>>(p);
+    else merge_kernel<false, kPassStats><<<p.R, kPassThreads, 0, s>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_pass_error(int* out) {

@@ -319,6 +319,17 @@ int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* 
 /* ------------------------------------------------------------------------ */
 int dg_test_bounded_wait(uint32_t limit_cycles, dg_stream_t stream);
 
+/* dg_test_merge_stall: the logits pass's per-row merge kernel alone (the   */
+/*   statistics epilogue), with nothing counting its rows: every row's wait */
+/*   gives up after limit_cycles (> 0), records device error 1, and the     */
+/*   merge finishes on whatever the workspace holds (lse is then            */
+/*   meaningless).  logits as dg_sampler_step with B = 1, C = rows; lse:    */
+/*   device float [rows]; workspace: dg_sampler_step_workspace_size(rows, V)*/
+/*   bytes, zeroed.                                                         */
+int dg_test_merge_stall(const void* logits, int logits_dtype, int64_t ld, int32_t rows, int32_t V,
+                        float* lse, void* workspace, size_t workspace_bytes, uint32_t limit_cycles,
+                        dg_stream_t stream);
+
 int dg_test_selfcond_stall(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C,
                            int32_t V, const float* inv_tau, const float* lse, const void* E,
                            int embed_dtype, int32_t d, void* z, void* workspace,

@@ -1,8 +1,8 @@
 """Failure detection on the GPU without a GPU fault.
 
 Every wait inside the library's kernels is bounded.  These tests make waits run out on purpose
--- a barrier nothing arrives on, and a contraction whose copy of one block of E is never
-issued -- and check that the kernels give up, report through dg_device_error() (code 1), free
+-- a barrier nothing arrives on, a contraction whose copy of one block of E is never issued, and
+per-row merges of the logits pass whose rows nothing counts -- and check that the kernels give up, report through dg_device_error() (code 1), free
 what they hold and leave the device usable: the next normal call gives the same result as a
 call made before the stall.  Limits are about 10 ms so the tests stay short.
 """
@@ -69,3 +69,26 @@ def test_contraction_stall_aborts_cleanly(name, block):
     torch.cuda.synchronize()
     assert dg.dg_device_error() == 0
     assert torch.equal(before, after)
+
+
+def test_merge_wait_gives_up_and_device_stays_usable():
+    cfg = W.TINY
+    logits = W.make_logits(cfg, "cuda")
+    x_t = W.make_canvas(cfg, "cuda")
+    R, V = logits.shape
+    nbytes = dg.dg_sampler_step_workspace_size(R, V)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    lse = torch.empty(R, dtype=torch.float32, device="cuda")
+    assert dg.dg_device_error() == 0
+    t0 = time.time()
+    rc = dg.lib().dg_test_merge_stall(ctypes.c_void_p(logits.data_ptr()), dg._dtype_code(logits), logits.stride(0),
+                                      R, V, ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(ws.data_ptr()), nbytes,
+                                      ctypes.c_uint32(LIMIT), _stream())
+    assert rc == 0, dg.dg_last_error()
+    assert dg.dg_device_error() == 1
+    assert time.time() - t0 < 5.0
+    # the device is usable and a normal step (on a fresh workspace) is right
+    out = dg.dg_sampler_step(logits, x_t, cfg.C, 0.5, 0.125, schedule="linear", mode="greedy")
+    torch.cuda.synchronize()
+    assert dg.dg_device_error() == 0
+    assert torch.equal(out["x0_hat"], logits.argmax(1).to(torch.int32))
