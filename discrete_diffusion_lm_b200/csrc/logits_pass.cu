@@ -284,7 +284,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             const long long t0 = clock64();
             const long long limit = p.merge_wait_limit > 0 ? p.merge_wait_limit : kMergeWaitLimit;
             while (ld_acquire(&p.row_count[row]) < target) {
-                __nanosleep(128);
+                __nanosleep(32);
                 if (clock64() - t0 > limit) {
                     atomicExch(&g_pass_error, 1);
                     break;
@@ -326,6 +326,13 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     int32_t xt = 0;
     unsigned long long thr_sd = 0, thr_jd = 0, thr_ss = 0;
     uint4 step_w = make_uint4(0u, 0u, 0u, 0u);
+    // output pointers, read from the parameter bank now rather than after the last exchange
+    int32_t* const out_x0 = p.x0_hat;
+    int32_t* const out_am = p.argmax;
+    float* const out_mp = p.max_prob;
+    float* const out_lse = p.lse;
+    float* const out_h = p.entropy;
+    if (kKind == kPassSampler && tid == 0) asm volatile("" ::"l"(out_x0), "l"(out_am), "l"(out_mp), "l"(out_lse), "l"(out_h));
     if (kKind == kPassSampler && tid == 0 && p.x_next) {
         xt = p.x_t[row];
         thr_sd = p.thr_stay_diff[canvas];
@@ -534,11 +541,11 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             p.x_next[row] = xn;
             if (p.branch) p.branch[row] = br;
         }
-        if (p.x0_hat) p.x0_hat[row] = x0;
-        if (p.argmax) p.argmax[row] = am;
-        if (p.max_prob) p.max_prob[row] = 1.0f / S;
-        if (p.lse) p.lse[row] = lse;
-        if (p.entropy) p.entropy[row] = ln_s - T / S;
+        if (out_x0) out_x0[row] = x0;
+        if (out_am) out_am[row] = am;
+        if (out_mp) out_mp[row] = 1.0f / S;
+        if (out_lse) out_lse[row] = lse;
+        if (out_h) out_h[row] = ln_s - T / S;
     }
 }
 
