@@ -433,7 +433,7 @@ int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, i
     sp.C = C;
     sp.V = V;
     sp.d = d;
-    // partial sums and tile tickets live at the end of the workspace
+    // the partial sums live at the end of the workspace
     sp.partial = reinterpret_cast<float*>(wp);
     sp.wait_limit = wait_limit;
     sp.fault_block = fault_block;

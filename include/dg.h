@@ -8,9 +8,13 @@
  *     the schedule kappa (monotone, kappa_0 = 1, kappa_1 = 0), the Step
  *     reverse transition, the per-iteration update
  *       p0 = Softmax(L_t / tau_t),  z = FFW(p0 E),  x_{t-dt} ~ Step(x_t, p0),
- *     and the canvas loss L = -sum_{i=1..C} log p(x_0^i | x_t, z_t, H);
+ *     the sampler paragraph (entropy-ordered acceptance under an error
+ *     tolerance with uniform re-noising, tau annealed linearly 0.8 -> 0.4,
+ *     adaptive stopping), and the canvas loss
+ *       L = -sum_{i=1..C} log p(x_0^i | x_t, z_t, H);
  *   section "Dataset" -- training sequences of P prompt tokens + K canvases of
- *     C tokens; the decoder loss on one canvas per sequence chosen uniformly.
+ *     C tokens; the decoder loss on one canvas per sequence chosen uniformly;
+ *     the self-conditioning state used for half of the batch, zero otherwise.
  *
  * Conventions shared by every entry point
  *   - Every function returns an int status (dg_status).  On failure nothing
@@ -28,7 +32,9 @@
  *     call; everything else named "device" is device memory.
  *   - All work is enqueued asynchronously on `stream` (a cudaStream_t;
  *     NULL = the legacy default stream).  Arguments are checked before any
- *     launch; the device work itself reports no errors.
+ *     launch.  Device-side waits are bounded: one that expires sets a device
+ *     error word read (and cleared) by dg_device_error(); re-zero the
+ *     workspace after such an error.
  *   - Logits rows: element (r, v) lives at logits + r*ld + v (elements), the
  *     base is 16-byte aligned and ld*sizeof(element) is a multiple of 16.
  *     Logits must be finite or -inf (a masked token); NaN is not supported.
@@ -39,6 +45,8 @@
  *       2 forward noise    (j, b, 0, 2): word 0 keep, word 1 token
  *       3 loss canvas      (0, b, 0, 3): word 0
  *       4 chunk Gumbel     (c >> 2, row, step, 4), word c & 3
+ *       5 re-noise         (0, row, step, 5): word 0 token (entropy-bounded)
+ *       6 self-cond drop   (0, b, step, 6): word 0 keep if < 2^31
  *     A word w becomes u = (2 (w >> 9) + 1) 2^-24 for a Gumbel variate
  *     -ln(-ln u), u = w 2^-32 for a comparison with a probability, and
  *     floor(w n / 2^32) for an index in [0, n).
