@@ -717,8 +717,22 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
     grid_dependency_wait();  // launched dependent on the contraction: its partials must be complete
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        // splits summed in order 0, 1, 2, ... (deterministic); loads issued eight at a time
         float4 acc = __ldcs(partial + i);
-        for (int s = 1; s < splits; ++s) {
+        int s = 1;
+        for (; s + 8 <= splits; s += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldcs(partial + static_cast<int64_t>(s + u) * n4 + i);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc.x += v[u].x;
+                acc.y += v[u].y;
+                acc.z += v[u].z;
+                acc.w += v[u].w;
+            }
+        }
+        for (; s < splits; ++s) {
             const float4 v = __ldcs(partial + static_cast<int64_t>(s) * n4 + i);
             acc.x += v.x;
             acc.y += v.y;
