@@ -111,7 +111,25 @@ def _check(fn: str, rc: int):
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor (None stays NULL).  Only CUDA tensors reach the library: a host
+    address handed to a kernel would fault the device."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("the library takes CUDA tensors only (got a tensor on %s)" % t.device)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _vec(t: Optional[torch.Tensor], name: str, dtype, n: Optional[int] = None):
+    """Check a contiguous device vector argument: dtype, and at least n elements when given."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if n is not None and t.numel() < n:
+        raise ValueError(f"{name} has {t.numel()} elements, {n} are needed")
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -185,6 +203,16 @@ def dg_canvas_ce_workspace_size(n_seq: int, C: int, V: int) -> int:
     return int(lib().dg_canvas_ce_workspace_size(n_seq, C, V))
 
 
+_STEP_OUT_DTYPES = {"x_next": torch.int32, "x0_hat": torch.int32, "argmax": torch.int32, "max_prob": torch.float32,
+                    "lse": torch.float32, "entropy": torch.float32, "branch": torch.uint8}
+
+
+def _check_step_vectors(x_t, out: dict, R: int):
+    _vec(x_t, "x_t", torch.int32, R)
+    for k, dt_ in _STEP_OUT_DTYPES.items():
+        _vec(out.get(k), k, dt_, R)
+
+
 def dg_sampler_step(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V: Optional[int] = None,
                     schedule: str = "cosine", inv_tau=None, seed: int = 0, step: int = 0, mode: str = "sample",
                     out: Optional[dict] = None, ws: Optional[torch.Tensor] = None, stream=None) -> dict:
@@ -207,6 +235,7 @@ def dg_sampler_step(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, dt, *, V
             "entropy": torch.empty(R, dtype=torch.float32, device=dev),
             "branch": torch.empty(R, dtype=torch.uint8, device=dev),
         }
+    _check_step_vectors(x_t, out, R)
     nbytes = dg_sampler_step_workspace_size(R, V)
     if ws is None:
         ws = workspace("sampler_step", nbytes, dev, (R, V), stream)
@@ -245,6 +274,8 @@ def dg_sampler_selfcond_step(logits: torch.Tensor, x_t: torch.Tensor, E: torch.T
                 ("branch", torch.uint8))}
     z = torch.empty((R, d), dtype=torch.bfloat16, device=dev) if z is None else z
     out["z"] = z
+    _check_step_vectors(x_t, out, R)
+    _vec(z, "z", torch.bfloat16, R * d)
     if ws is None:
         ws = workspace("sampler_step", dg_sampler_step_workspace_size(R, V), dev, (R, V), stream)
     if ws_z is None:
@@ -313,6 +344,8 @@ def dg_selfcond(logits: torch.Tensor, E: torch.Tensor, C: int, *, V: Optional[in
     dev = logits.device
     if z is None:
         z = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+    _vec(z, "z", torch.bfloat16, R * d)
+    _vec(lse, "lse", torch.float32, R)
     nbytes = dg_selfcond_workspace_size(R, V, d, _dtype_code(logits), _dtype_code(E), lse is not None)
     if ws is None:
         ws = workspace("selfcond", nbytes, dev, (R, V, d, lse is None, E.dtype), stream)
@@ -335,6 +368,8 @@ def dg_forward_noise(x0: torch.Tensor, P: int, K: int, C: int, V: int, t, *, sch
         x_t = torch.empty_like(x0)
     if canvas_idx is None:
         canvas_idx = torch.empty(n_seq, dtype=torch.int32, device=x0.device)
+    _vec(x_t, "x_t", torch.int32, x0.numel())
+    _vec(canvas_idx, "canvas_idx", torch.int32, n_seq)
     rc = lib().dg_forward_noise(_ptr(x0), n_seq, P, K, C, V, DG_SCHED[schedule],
                                 _host_doubles(_expand(t, n_seq), n_seq), ctypes.c_uint64(seed), _ptr(x_t),
                                 _ptr(canvas_idx), _stream(stream))
@@ -350,6 +385,8 @@ def dg_canvas_ce(logits: torch.Tensor, x0: torch.Tensor, canvas_idx: torch.Tenso
     R = logits.shape[0]
     V = logits.shape[1] if V is None else V
     n_seq = x0.shape[0]
+    _vec(x0, "x0", torch.int32)
+    _vec(canvas_idx, "canvas_idx", torch.int32, n_seq)
     if R != n_seq * C:
         raise ValueError("logits must have n_seq * C rows")
     dev = logits.device
@@ -385,6 +422,8 @@ def dg_entropy_accept(entropy: torch.Tensor, x0_hat: torch.Tensor, C: int, V: in
         raise ValueError("rows must be a multiple of C")
     B = R // C
     dev = entropy.device
+    _vec(entropy, "entropy", torch.float32)
+    _vec(x0_hat, "x0_hat", torch.int32, R)
     if out is None:
         out = {"x_next": torch.empty(R, dtype=torch.int32, device=dev),
                "accepted": torch.empty(R, dtype=torch.uint8, device=dev),
@@ -403,6 +442,9 @@ def dg_adaptive_stop(entropy: torch.Tensor, argmax: torch.Tensor, argmax_prev: O
     if R % C:
         raise ValueError("rows must be a multiple of C")
     B = R // C
+    _vec(entropy, "entropy", torch.float32)
+    _vec(argmax, "argmax", torch.int32, R)
+    _vec(argmax_prev, "argmax_prev", torch.int32, R)
     stop = torch.empty(B, dtype=torch.uint8, device=entropy.device)
     mean = torch.empty(B, dtype=torch.float32, device=entropy.device)
     rc = lib().dg_adaptive_stop(_ptr(entropy), _ptr(argmax), _ptr(argmax_prev), B, C, float(theta), _ptr(stop),
@@ -432,6 +474,7 @@ def dg_sampler_step_eb(logits: torch.Tensor, C: int, *, eps: float, theta: float
                 ("accepted", torch.uint8))}
         out["stop"] = torch.empty(B, dtype=torch.uint8, device=dev)
         out["mean_entropy"] = torch.empty(B, dtype=torch.float32, device=dev)
+    _vec(argmax_prev, "argmax_prev", torch.int32, R)
     nbytes = dg_sampler_step_workspace_size(R, V)
     if ws is None:
         ws = workspace("sampler_step", nbytes, dev, (R, V), stream)
@@ -454,6 +497,10 @@ def dg_canvas_ce_backward(logits: torch.Tensor, lse_rows: torch.Tensor, x0: torc
         raise TypeError("the in-place CE backward works on bf16 logits")
     V = logits.shape[1] if V is None else V
     n_seq = x0.shape[0]
+    _vec(lse_rows, "lse_rows", torch.float32, logits.shape[0])
+    _vec(x0, "x0", torch.int32)
+    _vec(canvas_idx, "canvas_idx", torch.int32, n_seq)
+    _vec(g_seq, "g_seq", torch.float32, n_seq)
     rc = lib().dg_canvas_ce_backward(_ptr(logits), ld, _ptr(lse_rows), _ptr(x0), _ptr(canvas_idx), n_seq, P, K, C, V,
                                      _ptr(g_seq), _stream(stream))
     _check("dg_canvas_ce_backward", rc)

@@ -174,3 +174,17 @@ def test_ffw_rejects(L):
     assert f(FAKE, 16, 64, 256, FAKE + 8, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 1 << 30, None) == 2
     assert f(FAKE, 16, 64, 256, FAKE, FAKE, FAKE, FAKE + 8192, FAKE, 1 << 30, None) == 1  # hidden aliases z_in
     assert f(FAKE, 256, 2048, 8192, FAKE, FAKE, FAKE + 4096, FAKE + 8192, FAKE, 8, None) == 3  # workspace
+
+
+def test_binding_rejects_host_and_mistyped_tensors(L):
+    # host tensors never reach the library; wrong dtypes are refused before any call
+    logits = torch.zeros(16, 1024, dtype=torch.bfloat16)
+    x_t = torch.zeros(16, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        dg.dg_sampler_step(logits, x_t, 16, 0.5, 0.1, ws=torch.zeros(1))
+    with pytest.raises(TypeError, match="x_t must be torch.int32"):
+        dg.dg_sampler_step(logits, x_t.long(), 16, 0.5, 0.1)
+    with pytest.raises(TypeError, match="entropy must be torch.float32"):
+        dg.dg_entropy_accept(torch.zeros(16, dtype=torch.float64), x_t, 16, 1024, 1.0)
+    with pytest.raises(TypeError, match="argmax_prev must be torch.int32"):
+        dg.dg_adaptive_stop(torch.zeros(16), x_t, x_t.long(), 16, 0.5)
