@@ -325,7 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 if (!mbar_wait(&efull[s], ph, wc)) break;
-                if (!mbar_wait(&pready[s], ph, wc)) break;
+                // plain operands are used as loaded: no softmax hand-off
+                if (!mbar_wait(p.plain ? &lfull[s] : &pready[s], ph, wc)) break;
                 tcgen05_after_sync();
                 uint8_t* st = smem + s * G::kStageBytes;
                 const uint32_t a_base = smem_u32(st + G::kEBytes + (kBf16 ? 0 : G::kLBytes));
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         const float a = it * kLog2e;
         grid_dependency_wait();  // lse comes from the preceding logits pass (a dependent launch)
         const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
-        for (int i = group; i < nkb; i += 2) {
+        for (int i = group; i < (p.plain ? 0 : nkb); i += 2) {  // plain operands need no softmax
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             const bool ok = mbar_wait(&lfull[s], ph, wc);
@@ -573,17 +574,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // ---------------------------------------------------------------- logits producer (both CTAs)
         if (lane == 0) {
             int issued = 0;
+            // Plain operands (bf16, used as loaded): both CTAs' tiles complete on the leader's barrier,
+            // which the MMA thread waits on directly.
+            const uint32_t leader_lfull0 = map_to_rank(smem_u32(&lfull[0]), 0);
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kLS;
                 const uint32_t ph = (i / kLS) & 1;
                 if (!mbar_wait(&lempty[s], ph ^ 1, wc)) break;
                 const int32_t k0 = (kb0 + i * kstride) * kKBlock;
-                mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
-                load_logits_tile<kBf16>(lring + s * G::kLStageBytes, &p.tm_logits, k0,
-                                        mp * 2 * kTileM + static_cast<int>(rank) * kTileM, &lfull[s]);
+                const int32_t row0 = mp * 2 * kTileM + static_cast<int>(rank) * kTileM;
+                if (kBf16 && p.plain) {
+                    if (rank == 0) mbar_arrive_expect_tx(&lfull[s], 2 * G::kLBytes);
+                    tma_load_2d_pair(lring + s * G::kLStageBytes, &p.tm_logits, k0, row0, leader_lfull0 + s * 8);
+                } else {
+                    mbar_arrive_expect_tx(&lfull[s], G::kLBytes);
+                    load_logits_tile<kBf16>(lring + s * G::kLStageBytes, &p.tm_logits, k0, row0, &lfull[s]);
+                }
                 issued = i + 1;
             }
-            if (aborted(wc)) {
+            if (aborted(wc) && (!p.plain || rank == 0)) {
                 const long long t0 = clock64();  // one deadline for the whole drain
                 for (int i = issued - kLS > 0 ? issued - kLS : 0; i < issued; ++i) {
                     while (!mbar_try_wait(&lfull[i % kLS], (i / kLS) & 1) && clock64() - t0 < wc->limit) {
@@ -596,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // Passes "p of stage s is written" on to the leader, off the softmax warps' critical path.
         if (lane == 0) {
             const uint32_t leader_pready0 = map_to_rank(smem_u32(&pready[0]), 0);
-            for (int i = 0; i < nkb; ++i) {
+            for (int i = 0; i < (p.plain ? 0 : nkb); ++i) {
                 const int s = i % kLS;
                 if (!mbar_wait(&pready[s], (i / kLS) & 1, wc)) break;
                 mbar_arrive_remote(leader_pready0 + s * 8);
@@ -613,7 +622,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int i = 0; i < nkb; ++i) {
                 const int es = i % kES, ls = i % kLS;
                 if (!mbar_wait(&efull[es], (i / kES) & 1, wc)) break;
-                if (!mbar_wait(&pready[ls], (i / kLS) & 1, wc)) break;
+                if (!mbar_wait(p.plain ? &lfull[ls] : &pready[ls], (i / kLS) & 1, wc)) break;
                 tcgen05_after_sync();
                 const uint32_t a_base = smem_u32(lring + ls * G::kLStageBytes + (kBf16 ? 0 : G::kLBytes));
                 const uint32_t b_base = smem_u32(ering + es * G::kEBytes);
@@ -648,7 +657,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         grid_dependency_wait();  // lse comes from the preceding logits pass (a dependent launch)
         const float nb = valid && !p.plain ? -p.lse[r] * kLog2e : 0.0f;
         const int leader_thread = (kFirstSoftmaxWarp + 4 * group) * 32;
-        for (int i = group; i < nkb; i += 2) {
+        for (int i = group; i < (p.plain ? 0 : nkb); i += 2) {  // plain operands need no softmax
             const int s = i % kLS;
             const bool ok = mbar_wait(&lfull[s], (i / kLS) & 1, wc);
             uint8_t* lt = lring + s * G::kLStageBytes;
