@@ -1,14 +1,35 @@
 """Python binding of libdg, the B200 (sm_100a) sampler library for block-parallel
-uniform-noise discrete diffusion (DiffusionGemma Technical Report, section "Method").
+uniform-noise discrete diffusion (DiffusionGemma Technical Report, sections "Method" and
+"Dataset").
 
 The binding only marshals arguments: torch tensors supply device memory and
 the current CUDA stream; every step of the computation runs in libdg's CUDA
-kernels.  There is no CPU fallback: if libdg.so is missing or the device is not
-sm_100, the calls raise.
+kernels.  There is no CPU fallback: if libdg.so is missing, a tensor is not on
+the GPU, or the device is not sm_100, the calls raise.
 
 Functions carry the C ABI's names (include/dg.h):
-    dg_sampler_step, dg_selfcond, dg_forward_noise, dg_canvas_ce
-plus the workspace-size queries, dg_last_error, dg_launch_count, dg_version.
+    sampler:   dg_sampler_step, dg_sampler_selfcond_step, dg_sampler_step_eb,
+               dg_entropy_accept, dg_adaptive_stop, dg_tau_linear, dg_sampler_step_noalloc
+    self-conditioning input:   dg_selfcond, dg_ffw
+    training:  dg_forward_noise, dg_canvas_ce, dg_canvas_ce_backward, dg_selfcond_drop
+plus the workspace-size queries, dg_last_error, dg_device_error, dg_launch_count, dg_version.
+
+Typical sampler loop over one 256-token canvas (logits from the model each step):
+
+    import discrete_diffusion_lm_b200 as dg
+    x = initial_canvas                                   # int32 [256] on the GPU
+    for k in range(steps):
+        t, dt = 1 - k / steps, 1 / steps
+        logits = model(x, z)                             # [256, V] bf16
+        out = dg.dg_sampler_selfcond_step(logits, x, E, 256, t, dt, step=k,
+                                          inv_tau=dg.dg_tau_linear([t]))
+        x, z = out["x_next"], out["z"]                   # next canvas, self-conditioning input
+
+or, with entropy-bounded acceptance and adaptive stopping instead of the Step posterior:
+
+        out = dg.dg_sampler_step_eb(logits, 256, eps=eps, theta=theta, argmax_prev=prev, step=k,
+                                    inv_tau=dg.dg_tau_linear([t]))
+        if out["stop"].item(): break
 """
 from __future__ import annotations
 
