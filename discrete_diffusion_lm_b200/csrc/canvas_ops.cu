@@ -9,17 +9,14 @@
 // Same page, section "Dataset": the self-conditioning state is used for half of the batch and
 //   zero for the other half.
 //
-// canvas_decide_kernel: one CTA of kDecideThreads threads per canvas (C <= DG_MAX_CANVAS_ROWS).
-//   Entropies become fixed-point integers q = floor(clamp(H, 0, 64) 2^32) (NaN -> 64), so sums
-//   and comparisons are exact and order-free.  Acceptance: ranks by (q, position) are computed by
-//   counting in shared memory, the rank-ordered q are prefix-summed (a block scan) and the
-//   accepted set is the ranks whose prefix is below the tolerance.  Stopping: the sum of q
-//   against the threshold, and an all-equal test of the argmax canvas against the previous one.
+// canvas_decide_kernel: one CTA of kDecideThreads threads per canvas (C <= DG_MAX_CANVAS_ROWS), the
+//   decisions of canvas_decide.cuh.
 // ce_backward_kernel: rows along grid y, 16-byte bf16 vectors of a row along grid x, in place.
 // selfcond_drop_kernel: sequences along grid y; a fair Philox coin per sequence decides, dropped
 //   rows are zeroed.
 #include <algorithm>
 
+#include "canvas_decide.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -28,125 +25,10 @@ namespace dg {
 namespace {
 
 constexpr int kDecideThreads = 256;
-constexpr int kPerThread = (DG_MAX_CANVAS_ROWS + kDecideThreads - 1) / kDecideThreads;
-
-__device__ __forceinline__ long long entropy_q(float h) {
-    float x = h;
-    if (!(x >= 0.f)) x = isnan(x) ? 64.f : 0.f;
-    x = fminf(x, 64.f);
-    return __float2ll_rd(x * 4294967296.f);  // exact: a power-of-two scale of a float
-}
-
-// Inclusive block-wide prefix sum of one 64-bit value per thread.
-__device__ __forceinline__ long long block_inclusive_scan(long long v, long long* sh_warp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const long long n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-    }
-    if (lane == 31) sh_warp[warp] = v;
-    __syncthreads();
-    long long base = 0;
-    for (int w = 0; w < warp; ++w) base += sh_warp[w];
-    __syncthreads();
-    return v + base;
-}
 
 __global__ void __launch_bounds__(kDecideThreads) canvas_decide_kernel(const __grid_constant__ DecideParams p) {
-    __shared__ long long q[DG_MAX_CANVAS_ROWS];
-    __shared__ long long sorted[DG_MAX_CANVAS_ROWS];
-    __shared__ long long sh_warp[kDecideThreads / 32];
-    __shared__ int sh_count[kDecideThreads / 32];
-    __shared__ int sh_same;
-    const int b = blockIdx.x, tid = threadIdx.x;
-    const int C = p.C;
-    const int64_t r0 = static_cast<int64_t>(b) * C;
-    if (tid == 0) sh_same = 1;
-    for (int i = tid; i < C; i += kDecideThreads) q[i] = entropy_q(p.entropy[r0 + i]);
-    __syncthreads();
-
-    // ---- adaptive stopping: sum of q and the argmax comparison
-    if (p.stop || p.mean_entropy) {
-        long long s = 0;
-        int diff = 0;
-        for (int i = tid; i < C; i += kDecideThreads) {
-            s += q[i];
-            if (p.argmax_prev && p.argmax[r0 + i] != p.argmax_prev[r0 + i]) diff = 1;
-        }
-        if (__any_sync(0xffffffffu, diff) && (tid & 31) == 0) sh_same = 0;
-        const long long total = block_inclusive_scan(s, sh_warp);  // the last thread holds the sum
-        if (tid == kDecideThreads - 1) {
-            const bool same = p.argmax_prev != nullptr && sh_same != 0;
-            if (p.stop) p.stop[b] = static_cast<uint8_t>(total < p.stop_limit && same);
-            if (p.mean_entropy)
-                p.mean_entropy[b] = static_cast<float>(static_cast<double>(total) * (1.0 / 4294967296.0) /
-                                                       static_cast<double>(C));
-        }
-    }
-    if (!p.x_next) return;
-
-    // ---- entropy-bounded acceptance
-    int rank[kPerThread];
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int i = tid + u * kDecideThreads;
-        rank[u] = 0;
-        if (i < C) {
-            const long long qi = q[i];
-            int r = 0;
-            for (int j = 0; j < C; ++j) {
-                const long long qj = q[j];
-                r += (qj < qi) | ((qj == qi) & (j < i));
-            }
-            rank[u] = r;
-            sorted[r] = qi;
-        }
-    }
-    __syncthreads();
-    // thread t scans ranks kPerThread t .. kPerThread t + kPerThread - 1
-    long long local[kPerThread];
-    long long run = 0;
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int k = tid * kPerThread + u;
-        run += k < C ? sorted[k] : 0;
-        local[u] = run;
-    }
-    const long long incl = block_inclusive_scan(run, sh_warp);
-    const long long base = incl - run;
-    int cnt = 0;
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int k = tid * kPerThread + u;
-        cnt += (k < C) & (base + local[u] < p.accept_limit);
-    }
-    // the accepted ranks are a prefix (q >= 0): their number is the count of passing prefixes
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if ((tid & 31) == 0) sh_count[tid >> 5] = cnt;
-    __syncthreads();
-    int n_acc = 0;
-#pragma unroll
-    for (int w = 0; w < kDecideThreads / 32; ++w) n_acc += sh_count[w];
-    if (tid == 0 && p.n_accepted) p.n_accepted[b] = n_acc;
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int i = tid + u * kDecideThreads;
-        if (i < C) {
-            const int64_t r = r0 + i;
-            const bool acc = rank[u] < n_acc;
-            int32_t x;
-            if (acc) {
-                x = p.x0_hat[r];
-            } else {
-                const uint4 w = philox4x32_10(
-                    make_uint4(0u, static_cast<uint32_t>(r), p.step, kDomRenoise), p.key0, p.key1);
-                x = word_to_index(w.x, p.V);
-            }
-            p.x_next[r] = x;
-            if (p.accepted) p.accepted[r] = static_cast<uint8_t>(acc);
-        }
-    }
+    __shared__ DecideShared sh;
+    decide_canvas<kDecideThreads>(p, blockIdx.x, sh);
 }
 
 // grad = g_seq[b] (exp(l - lse) - [v == y]) over bf16 rows, in place.  Grid: x covers a row's

@@ -99,6 +99,28 @@ def test_sampler_step_eb_equals_its_parts():
         assert torch.equal(fused[k], plain[k]), k
 
 
+def test_sampler_step_eb_batched_equals_its_parts():
+    # 16 canvases with per-canvas temperatures: the decisions run in the merge of each canvas's
+    # last row and must equal the standalone decisions on the same outputs
+    cfg = W.BATCHED
+    rows = 16 * 256
+    logits = W.make_logits(cfg, DEV, rows=rows)
+    ts = [1.0 - b / 16 for b in range(16)]
+    inv_tau = dg.dg_tau_linear(ts)
+    prev = torch.from_numpy(np.random.default_rng(1).integers(0, cfg.V, rows).astype(np.int32)).to(DEV)
+    for rep in range(2):  # the canvas tickets must be back at zero for the second call
+        fused = dg.dg_sampler_step_eb(logits, cfg.C, eps=40.0, theta=6.0, argmax_prev=prev, inv_tau=inv_tau, seed=7,
+                                      step=5 + rep)
+        torch.cuda.synchronize()
+        acc = dg.dg_entropy_accept(fused["entropy"], fused["x0_hat"], cfg.C, cfg.V, 40.0, seed=7, step=5 + rep)
+        stop, mean = dg.dg_adaptive_stop(fused["entropy"], fused["argmax"], prev, cfg.C, 6.0)
+        torch.cuda.synchronize()
+        assert torch.equal(fused["x_next"], acc["x_next"]) and torch.equal(fused["accepted"], acc["accepted"])
+        assert torch.equal(fused["stop"], stop) and torch.equal(fused["mean_entropy"], mean)
+        prev = fused["argmax"].clone()
+    assert dg.dg_device_error() == 0
+
+
 @pytest.mark.parametrize("mode", ["sample", "greedy"])
 def test_sampler_step_eb_vs_oracle_mid(mode):
     cfg = W.MID
