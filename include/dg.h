@@ -69,7 +69,7 @@ typedef enum dg_status {
     DG_ERR_ALIGNMENT = 2,   /* a pointer or leading dimension breaks the 16-byte rule */
     DG_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query */
     DG_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
-    DG_ERR_UNSUPPORTED = 5  /* valid request this build does not handle (e.g. no sm_100 device) */
+    DG_ERR_UNSUPPORTED = 5  /* valid request the library does not handle (e.g. no sm_100 device) */
 } dg_status;
 
 typedef enum dg_dtype { DG_F32 = 0, DG_BF16 = 1 } dg_dtype;
