@@ -18,11 +18,11 @@ Also reported: the dominant kernel's roofline (measured peaks), an end-to-end fi
 through the public API with host buffers (host->device logits copy and device->host read
 of x_next and z inside the timed region), the training-side kernels (forward noise and
 canvas cross-entropy on the training workload), the CPU oracle timed on a bounded sample
-(rank 0, N = 1), SM clocks sampled during the timed region, and the number of library
-kernel launches in the timed region.
+(rank 0, N = 1; on one thread, and over row blocks on every host core), SM clocks sampled
+during the timed region, and the number of library kernel launches in the timed region.
 
 --impl reference times the CPU oracle (the plain C reference of the same computation) on a
-bounded sample of the same workload, on the host's cores.
+bounded sample of the same workload, on one host core.
 """
 from __future__ import annotations
 
@@ -592,15 +592,15 @@ def bench_e2e(dg, W, cfg, dev, E, args, world, barrier, stream):
 
 # ------------------------------------------------------------------------------ the oracle
 class OracleSample:
-    """The CPU oracle (plain single-threaded C, double precision, as it stands) on a bounded sample
-    of the full-vocab workload: the logits-pass work (statistics, argmax, two-level draw, Step)
-    on `rows1` rows and the contraction z = softmax(l) E on `rows2` rows over a fraction
-    `vfrac` of the vocabulary; the measured time is scaled to one step (256 rows, all of V)."""
+    """The CPU oracle (plain C, double precision, as it stands) on a bounded sample of the
+    full-vocab workload: the logits-pass work (statistics, argmax, two-level draw, Step) on
+    `rows1` rows and the contraction z = softmax(l) E on `rows2` rows over a fraction `vfrac` of
+    the vocabulary; the measured time is scaled to one step (256 rows, all of V)."""
 
-    def __init__(self, rows1: int, rows2: int, vfrac: int):
+    def __init__(self, rows1: int, rows2: int, vfrac: int, cfg=None):
         import numpy as np
         from discrete_diffusion_lm_b200 import workloads as W
-        self.cfg = cfg = W.FULL
+        self.cfg = cfg = cfg or W.FULL
         self.rows1, self.rows2, self.vfrac = rows1, rows2, vfrac
         n = max(rows1, rows2)
         self.L = W.make_logits(cfg, "cpu", rows=n).float().numpy()
@@ -609,28 +609,82 @@ class OracleSample:
         self.Ls = np.ascontiguousarray(self.L[:rows2, : self.Vs])
         self.x_t = np.zeros(rows1, dtype=np.int32)
 
-    def run(self) -> dict:
+    def _pass(self, a: int, b: int):
         from oracle import oracle as O
         cfg = self.cfg
         t, dt = cfg.times(0)
-        t0 = time.perf_counter()
-        O.sampler_step(self.L[: self.rows1], self.x_t, 1, self.rows1, cfg.V, cfg.schedule, t[:1], dt[:1], None, 0, 0,
+        O.sampler_step(self.L[a:b], self.x_t[a:b], 1, b - a, cfg.V, cfg.schedule, t[:1], dt[:1], None, 0, 0,
                        "sample")
+
+    def _z(self, a: int, b: int):
+        from oracle import oracle as O
+        O.selfcond_rows(self.Ls, self.E, list(range(a, b)))
+
+    def _what(self) -> str:
+        c = self.cfg
+        return f"{c.name} workload (C={c.C}, V={c.V}, d={c.d})"
+
+    def _per_step(self, t_pass: float, rows1: int, t_z: float, rows2: int) -> float:
+        return self.cfg.R * (t_pass / rows1 + t_z * self.vfrac / rows2)
+
+    def run(self, rows2: int = 0) -> dict:
+        """Single thread: the logits pass on all `rows1` rows, z on the first `rows2` rows."""
+        rows2 = rows2 or self.rows2
+        t0 = time.perf_counter()
+        self._pass(0, self.rows1)
         t1 = time.perf_counter()
-        O.selfcond_rows(self.Ls, self.E, list(range(self.rows2)))
+        self._z(0, rows2)
         t2 = time.perf_counter()
-        step_s = cfg.R * ((t1 - t0) / self.rows1 + (t2 - t1) * self.vfrac / self.rows2)
+        step_s = self._per_step(t1 - t0, self.rows1, t2 - t1, rows2)
         return {"value": 1.0 / step_s, "unit": "steps/s", "cores": 1, "kind": "oracle", "cpu_seconds": t2 - t0,
-                "sample": f"full-vocab workload: logits pass on {self.rows1} rows of V=262144 + z on "
-                          f"{self.rows2} rows over 1/{self.vfrac} of V, scaled to 256 rows x full V per step"}
+                "sample": f"{self._what()}: logits pass on {self.rows1} rows + z on {rows2} rows over "
+                          f"1/{self.vfrac} of V, scaled to {self.cfg.R} rows x full V per step"}
+
+    def run_threads(self, threads: int) -> dict:
+        """The same routines over contiguous row blocks, one block per thread, all threads at once
+        (the C oracle keeps no global state, and ctypes releases the GIL for each foreign call).
+        A block restarts the oracle's row numbering, which changes the random words drawn, not
+        the work done."""
+        from concurrent.futures import ThreadPoolExecutor
+
+        def blocks(n):
+            k = min(threads, n)
+            edges = [n * i // k for i in range(k + 1)]
+            return list(zip(edges[:-1], edges[1:]))
+
+        with ThreadPoolExecutor(max_workers=threads) as pool:
+            t0 = time.perf_counter()
+            list(pool.map(lambda ab: self._pass(*ab), blocks(self.rows1)))
+            t1 = time.perf_counter()
+            list(pool.map(lambda ab: self._z(*ab), blocks(self.rows2)))
+            t2 = time.perf_counter()
+        step_s = self._per_step(t1 - t0, self.rows1, t2 - t1, self.rows2)
+        return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                "cpu_seconds": t2 - t0,
+                "sample": f"{self._what()}: logits pass on {self.rows1} rows + z on {self.rows2} rows over "
+                          f"1/{self.vfrac} of V, split into row blocks over {threads} threads, scaled to "
+                          f"{self.cfg.R} rows x full V per step"}
 
 
-def oracle_baseline() -> dict:
-    """About 10-20 s of single-threaded oracle work on rank 0."""
-    r = OracleSample(rows1=256, rows2=24, vfrac=1).run()
-    r["value"] = round(r["value"], 6)
-    r["cpu_seconds"] = round(r["cpu_seconds"], 1)
-    return r
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_baseline() -> tuple:
+    """About 10-20 s of single-threaded oracle work on rank 0, then the same routines on every
+    host core (z on up to three rows per thread, at most all 256)."""
+    cores = host_cores()
+    single_rows2 = 24
+    samp = OracleSample(rows1=256, rows2=min(256, max(single_rows2, 3 * cores)), vfrac=1)
+    one = samp.run(rows2=single_rows2)
+    many = samp.run_threads(cores)
+    for r in (one, many):
+        r["value"] = round(r["value"], 6)
+        r["cpu_seconds"] = round(r["cpu_seconds"], 1)
+    return one, many
 
 
 def run_reference(args, rank, world):
@@ -678,7 +732,7 @@ def main():
                                              timeout=__import__("datetime").timedelta(seconds=120))
     line = run_ours(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_baseline()
+        line["cpu_baseline"], line["cpu_baseline_all_cores"] = oracle_baseline()
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -49,3 +49,30 @@ def test_clock_summary_parses_samples():
     assert s["reasons"] == ["sw_power_cap"]
     empty = bench.ClockSampler(0)
     assert empty.summary()["samples"] == 0
+
+
+def test_oracle_sample_single_and_threaded_on_tiny():
+    from discrete_diffusion_lm_b200 import workloads as W
+    samp = bench.OracleSample(rows1=16, rows2=16, vfrac=1, cfg=W.TINY)
+    one = samp.run(rows2=4)
+    many = samp.run_threads(3)  # 16 rows over 3 threads: ragged blocks of 5, 5, 6
+    assert one["cores"] == 1 and many["cores"] == 3
+    assert one["value"] > 0 and many["value"] > 0
+    assert "tiny workload" in one["sample"] and "3 threads" in many["sample"]
+    more_threads_than_rows = samp.run_threads(40)
+    assert more_threads_than_rows["value"] > 0
+
+
+def test_reference_arm_prints_one_json_line():
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                         cwd=bench.ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "steps/s" and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["value"] == rec["value"]
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["warmup"] >= 3
