@@ -666,11 +666,19 @@ class OracleSample:
                           f"{self.cfg.R} rows x full V per step"}
 
 
-def host_cores() -> int:
+def host_cores(cpu_max_path: str = "/sys/fs/cgroup/cpu.max") -> int:
+    """Cores this process may run on: its affinity mask, capped by a cgroup CPU quota if any."""
     try:
-        return len(os.sched_getaffinity(0))
+        n = len(os.sched_getaffinity(0))
     except AttributeError:
-        return os.cpu_count() or 1
+        n = os.cpu_count() or 1
+    try:
+        quota, period = open(cpu_max_path).read().split()[:2]
+        if quota != "max":
+            n = min(n, max(1, math.ceil(int(quota) / int(period))))
+    except (OSError, ValueError):
+        pass
+    return n
 
 
 def oracle_baseline() -> tuple:

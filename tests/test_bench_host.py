@@ -76,3 +76,13 @@ def test_reference_arm_prints_one_json_line():
     assert rec["impl"] == "reference" and rec["unit"] == "steps/s" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["value"] == rec["value"]
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["warmup"] >= 3
+
+
+def test_host_cores_honours_a_cgroup_quota(tmp_path):
+    f = tmp_path / "cpu.max"
+    f.write_text("max 100000\n")
+    free = bench.host_cores(str(f))
+    assert free >= 1
+    f.write_text("150000 100000\n")  # 1.5 CPUs of quota -> 2 threads at most
+    assert bench.host_cores(str(f)) == min(free, 2)
+    assert bench.host_cores(str(tmp_path / "absent")) == free
