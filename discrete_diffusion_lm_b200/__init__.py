@@ -48,6 +48,8 @@ DG_SCHED = {"linear": 0, "cosine": 1}
 DG_X0 = {"sample": 0, "greedy": 1}
 DG_GUMBEL_CHUNK = 512
 DG_MAX_CANVASES = 256
+DG_MAX_CANVAS_ROWS = 1024
+DG_MAX_VOCAB = 1 << 30
 
 
 class DGError(RuntimeError):

@@ -140,6 +140,7 @@ int check_logits(const void* logits, int dtype, int64_t ld, int32_t V) {
     if (!logits) return fail(DG_ERR_INVALID_ARG, "logits is NULL");
     if (!valid_dtype(dtype)) return fail(DG_ERR_INVALID_ARG, "logits dtype %d is not DG_F32 or DG_BF16", dtype);
     if (V < 1) return fail(DG_ERR_INVALID_ARG, "V = %d must be >= 1", V);
+    if (V > DG_MAX_VOCAB) return fail(DG_ERR_INVALID_ARG, "V = %d exceeds DG_MAX_VOCAB = %d", V, DG_MAX_VOCAB);
     if (ld < V) return fail(DG_ERR_INVALID_ARG, "ld = %lld is smaller than V = %d", (long long)ld, V);
     if (!aligned16(logits)) return fail(DG_ERR_ALIGNMENT, "logits base is not 16-byte aligned");
     if ((ld * elt_size(dtype)) % 16 != 0)

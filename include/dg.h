@@ -91,6 +91,7 @@ typedef enum dg_x0_mode { DG_X0_SAMPLE = 0, DG_X0_GREEDY = 1 } dg_x0_mode;
 #define DG_GUMBEL_CHUNK 512
 #define DG_MAX_CANVASES 256 /* canvases (B, n_seq) per call */
 #define DG_MAX_CANVAS_ROWS 1024 /* C for the per-canvas decisions (acceptance, stopping) */
+#define DG_MAX_VOCAB (1 << 30) /* V for every call that reads logits rows (ids stay in 32 bits with headroom) */
 
 /* Human-readable reason for the last failure on this thread ("" if none). */
 const char* dg_last_error(void);
@@ -122,7 +123,7 @@ int dg_device_error(int* code);
 /* inv_tau: host float [B] (> 0, finite) or NULL for 1.                      */
 /* Outputs (device, [B*C]): x_next int32 (required); x0_hat, argmax int32,   */
 /* max_prob, lse, entropy float32, branch uint8 -- each may be NULL.         */
-/* 1 <= B <= DG_MAX_CANVASES, C >= 1, 1 <= V < 2^31, B*C < 2^31.             */
+/* 1 <= B <= DG_MAX_CANVASES, C >= 1, 1 <= V <= DG_MAX_VOCAB, B*C < 2^31.   */
 /* ------------------------------------------------------------------------ */
 size_t dg_sampler_step_workspace_size(int32_t rows, int32_t V);
 

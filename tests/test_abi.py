@@ -59,6 +59,7 @@ def _step(L, **kw):
     (dict(logits=None), 1, "logits is NULL"),
     (dict(dtype=7), 1, "dtype"),
     (dict(V=0), 1, "V = 0"),
+    (dict(V=(1 << 30) + 8, ld=(1 << 30) + 8), 1, "DG_MAX_VOCAB"),
     (dict(ld=1000), 1, "smaller than V"),
     (dict(logits=FAKE + 2), 2, "16-byte"),
     (dict(ld=1028, V=1025), 2, "multiple of 16"),
@@ -188,3 +189,26 @@ def test_binding_rejects_host_and_mistyped_tensors(L):
         dg.dg_entropy_accept(torch.zeros(16, dtype=torch.float64), x_t, 16, 1024, 1.0)
     with pytest.raises(TypeError, match="argmax_prev must be torch.int32"):
         dg.dg_adaptive_stop(torch.zeros(16), x_t, x_t.long(), 16, 0.5)
+
+
+def _int_expr(src: str) -> int:
+    """Value of a #define body made of integer literals, *, << and parentheses."""
+    import ast
+    import operator
+    ops = {ast.Mult: operator.mul, ast.LShift: operator.lshift}
+
+    def ev(n):
+        if isinstance(n, ast.Constant) and isinstance(n.value, int):
+            return n.value
+        if isinstance(n, ast.BinOp) and type(n.op) in ops:
+            return ops[type(n.op)](ev(n.left), ev(n.right))
+        raise ValueError(src)
+    return ev(ast.parse(src.strip(), mode="eval").body)
+
+
+def test_binding_constants_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    defines = {name: body for name, body in re.findall(r"#define\s+(DG_[A-Z_]+)[ \t]+([^\n]+)", text)}
+    for name in ("DG_GUMBEL_CHUNK", "DG_MAX_CANVASES", "DG_MAX_CANVAS_ROWS", "DG_MAX_VOCAB",
+                 "DG_NOALLOC_SCRATCH_BYTES"):
+        assert getattr(dg, name) == _int_expr(defines[name]), name

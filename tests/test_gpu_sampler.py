@@ -131,6 +131,28 @@ def test_edge_shapes(V, ld, C, B, dtype):
         check_sampler(out, ref, mode, label=f"V={V} ld={ld} C={C} B={B} {dtype}")
 
 
+@pytest.mark.parametrize("V", [262144 + 6 * 512 + 5, 1 << 20])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_rows_longer_than_512_chunks(V, dtype):
+    # past 512 chunks the merge keeps the first 512 records in registers and re-reads the rest
+    B, C = 2, 3
+    R, ld = B * C, (V + 7) // 8 * 8
+    g = torch.Generator(device=DEV).manual_seed(V)
+    full = torch.zeros((R, ld), device=DEV, dtype=torch.float32)
+    full[:, :V] = torch.randn((R, V), device=DEV, generator=g) * 2
+    full[0, V - 1] = 14.0  # the row maximum in the last (ragged) chunk
+    full[1, 600 * 512 + 9] = 14.0  # ... in a chunk past the first 512
+    full[2, :V] = 0.5  # a constant row: argmax 0
+    logits = full.to(dtype)
+    x_t = torch.randint(0, V, (R,), device=DEV, dtype=torch.int32, generator=g)
+    for mode in ("sample", "greedy"):
+        out, ref = run_both(logits, x_t, C, [0.7, 0.3], [0.1, 0.3], schedule="cosine", seed=9, step=4, mode=mode,
+                            V=V)
+        check_sampler(out, ref, mode, label=f"V={V} {dtype}")
+    assert int(out["argmax"][0]) == V - 1 and int(out["argmax"][1]) == 600 * 512 + 9
+    assert int(out["argmax"][2]) == 0
+
+
 def test_masked_logits_and_ties():
     V, C = 3000, 8
     g = torch.Generator(device=DEV).manual_seed(1)

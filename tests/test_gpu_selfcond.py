@@ -101,6 +101,7 @@ def test_batched_sampled_rows_and_mass():
     (64, 64, 777, 784, 256, torch.bfloat16, torch.float32),
     (129, 43, 3000, 3000, 1536, torch.bfloat16, torch.bfloat16),
     (1, 1, 33, 40, 512, torch.float32, torch.float32),
+    (6, 3, (1 << 20) + 3, (1 << 20) + 8, 64, torch.bfloat16, torch.bfloat16),  # rows past 512 chunks
 ])
 def test_edge_shapes(R, C, V, ld, d, ldt, edt):
     g = torch.Generator(device=DEV).manual_seed(R + V + d)

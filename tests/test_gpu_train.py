@@ -82,6 +82,24 @@ def test_canvas_ce_small_exact_and_torch(dtype):
     torch.testing.assert_close(loss.double(), ref, atol=1e-3, rtol=1e-5)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_canvas_ce_rows_longer_than_512_chunks(dtype):
+    n_seq, P, K, C, V = 2, 3, 2, 3, 262144 + 8 * 512 + 3
+    g = torch.Generator(device=DEV).manual_seed(3)
+    x0 = torch.randint(0, V, (n_seq, P + K * C), device=DEV, dtype=torch.int32, generator=g)
+    x0[0, P] = V - 1  # a target in the last, ragged chunk
+    kidx = torch.tensor([0, 1], device=DEV, dtype=torch.int32)
+    padded = torch.zeros((n_seq * C, V + 5), device=DEV, dtype=dtype)
+    logits = padded[:, :V]
+    logits.copy_((torch.randn((n_seq * C, V), device=DEV, generator=g) * 2).to(dtype))
+    loss, seq, lse = dg_canvas_ce(logits, x0, kidx, P, K, C)
+    torch.cuda.synchronize()
+    rl, rs, rlse = O.canvas_ce(host_f32(logits), x0.cpu().numpy(), kidx.cpu().numpy(), n_seq, P, K, C, V)
+    assert np.all(np.abs(loss.cpu().numpy() - rl) <= 1e-3 + 1e-5 * np.abs(rl))
+    assert np.all(np.abs(lse.cpu().numpy() - rlse) <= 1e-3)
+    np.testing.assert_allclose(seq.cpu().numpy(), rs, rtol=1e-5, atol=1e-3)
+
+
 def test_canvas_ce_bad_target_gives_nan_not_fault():
     n_seq, P, K, C, V = 2, 1, 2, 4, 100
     x0 = torch.zeros((n_seq, P + K * C), device=DEV, dtype=torch.int32)
