@@ -141,7 +141,8 @@ def test_rows_longer_than_512_chunks(V, dtype):
     full = torch.zeros((R, ld), device=DEV, dtype=torch.float32)
     full[:, :V] = torch.randn((R, V), device=DEV, generator=g) * 2
     full[0, V - 1] = 14.0  # the row maximum in the last (ragged) chunk
-    full[1, 600 * 512 + 9] = 14.0  # ... in a chunk past the first 512
+    far = (V // 512 - 2) * 512 + 9  # ... in a chunk past the first 512
+    full[1, far] = 14.0
     full[2, :V] = 0.5  # a constant row: argmax 0
     logits = full.to(dtype)
     x_t = torch.randint(0, V, (R,), device=DEV, dtype=torch.int32, generator=g)
@@ -149,7 +150,7 @@ def test_rows_longer_than_512_chunks(V, dtype):
         out, ref = run_both(logits, x_t, C, [0.7, 0.3], [0.1, 0.3], schedule="cosine", seed=9, step=4, mode=mode,
                             V=V)
         check_sampler(out, ref, mode, label=f"V={V} {dtype}")
-    assert int(out["argmax"][0]) == V - 1 and int(out["argmax"][1]) == 600 * 512 + 9
+    assert int(out["argmax"][0]) == V - 1 and int(out["argmax"][1]) == far
     assert int(out["argmax"][2]) == 0
 
 
