@@ -97,8 +97,9 @@ def make_logits(cfg: SamplerConfig, device="cpu", rows: int | None = None, seed:
             whose values are *set* to U[8, 12].
     zipf64: background N(0, std); on 64 distinct random ids per row a boost
             12 - 1.1 ln k (k = 1..64) is *added*: the log of a Zipf(s = 1.1)
-            profile over the top-64 set, offset so the set holds about half of
-            the probability mass.
+            profile over the top-64 set.  With std = 1.5 the set holds about
+            70% of a row's probability mass (0.71 in expectation, since the
+            background lifts each boosted id by e^{std^2 / 2} on average).
     """
     R = cfg.R if rows is None else rows
     V = cfg.V
