@@ -86,3 +86,33 @@ def test_host_cores_honours_a_cgroup_quota(tmp_path):
     f.write_text("150000 100000\n")  # 1.5 CPUs of quota -> 2 threads at most
     assert bench.host_cores(str(f)) == min(free, 2)
     assert bench.host_cores(str(tmp_path / "absent")) == free
+
+
+def test_oracle_routines_give_the_same_results_from_threads():
+    # the all-cores timings call the C oracle from several threads at once: each call must depend
+    # only on its own arguments
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    from discrete_diffusion_lm_b200 import workloads as W
+    from oracle import oracle as O
+    cfg = W.TINY
+    L = W.make_logits(cfg, "cpu").numpy()
+    E = W.make_embedding(cfg, "cpu").numpy()
+    x_t = W.make_canvas(cfg, "cpu").numpy()
+    t, dt = cfg.times(2)
+
+    def step(r):
+        return O.sampler_step(L[r:r + 1], x_t[r:r + 1], 1, 1, cfg.V, cfg.schedule, t, dt, None, 7, 2, "sample")
+
+    def z(r):
+        return O.selfcond_rows(L, E, [r])
+
+    serial = [step(r) for r in range(cfg.R)], [z(r) for r in range(cfg.R)]
+    with ThreadPoolExecutor(max_workers=8) as pool:
+        threaded = list(pool.map(step, range(cfg.R))), list(pool.map(z, range(cfg.R)))
+    for a, b in zip(serial[0], threaded[0]):
+        for k in ("x_next", "x0_hat", "argmax", "lse", "entropy"):
+            assert np.array_equal(a[k], b[k]), k
+    for a, b in zip(serial[1], threaded[1]):
+        assert np.array_equal(a, b)
