@@ -340,6 +340,7 @@ def dg_sampler_step_noalloc(logits: torch.Tensor, x_t: torch.Tensor, C: int, t, 
                (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32),
                 ("max_prob", torch.float32), ("lse", torch.float32), ("entropy", torch.float32),
                 ("branch", torch.uint8))}
+    _check_step_vectors(x_t, out, R)
     rc = lib().dg_sampler_step_noalloc(
         _ptr(logits), _dtype_code(logits), ld, _ptr(x_t), B, C, V, DG_SCHED[schedule],
         _host_doubles(_expand(t, B), B), _host_doubles(_expand(dt, B), B),

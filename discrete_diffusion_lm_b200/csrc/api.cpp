@@ -209,6 +209,23 @@ int dg_sampler_step(const void* logits, int logits_dtype, int64_t ld, const int3
                     uint32_t step, int x0_mode, int32_t* x_next, int32_t* x0_hat, int32_t* argmax, float* max_prob,
                     float* lse, float* entropy, uint8_t* branch, void* workspace, size_t workspace_bytes,
                     dg_stream_t stream) {
+    return dg::sampler_step_impl(logits, logits_dtype, ld, x_t, B, C, V, schedule, t, dt, inv_tau, seed, step, x0_mode,
+                                 x_next, x0_hat, argmax, max_prob, lse, entropy, branch, workspace, workspace_bytes,
+                                 stream, false);
+}
+
+}  // extern "C"
+
+namespace dg {
+
+// The sampler step behind dg_sampler_step and dg_sampler_step_noalloc.  Every argument is checked
+// before anything is enqueued; with clear_ws the workspace is zeroed on the stream (after the
+// checks, right before the launches).
+int sampler_step_impl(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t, int32_t B, int32_t C,
+                      int32_t V, int schedule, const double* t, const double* dt, const float* inv_tau, uint64_t seed,
+                      uint32_t step, int x0_mode, int32_t* x_next, int32_t* x0_hat, int32_t* argmax, float* max_prob,
+                      float* lse, float* entropy, uint8_t* branch, void* workspace, size_t workspace_bytes,
+                      dg_stream_t stream, bool clear_ws) {
     g_last_error.clear();
     int rc;
     if ((rc = check_logits(logits, logits_dtype, ld, V)) != DG_OK) return rc;
@@ -259,10 +276,18 @@ int dg_sampler_step(const void* logits, int logits_dtype, int64_t ld, const int3
     p.lse = lse;
     p.entropy = entropy;
     p.branch = branch;
+    if (clear_ws) {
+        const cudaError_t z = cudaMemsetAsync(workspace, 0, need, reinterpret_cast<cudaStream_t>(stream));
+        if (z != cudaSuccess) return cuda_fail(z, "workspace clear");
+    }
     const cudaError_t e = launch_logits_pass(p, kPassSampler, logits_dtype == DG_BF16, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "logits pass launch");
     return DG_OK;
 }
+
+}  // namespace dg
+
+extern "C" {
 
 int dg_forward_noise(const int32_t* x0, int32_t n_seq, int32_t P, int32_t K, int32_t C, int32_t V, int schedule,
                      const double* t, uint64_t seed, int32_t* x_t, int32_t* canvas_idx, dg_stream_t stream) {

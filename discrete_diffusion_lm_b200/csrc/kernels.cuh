@@ -137,6 +137,15 @@ cudaError_t launch_ce_backward(const CeBackwardParams& p, cudaStream_t s);
 cudaError_t launch_selfcond_drop(uint16_t* z, int32_t n_seq, int64_t seq_elems, uint32_t key0, uint32_t key1,
                                  uint32_t step, uint8_t* keep, cudaStream_t s);
 
+// The sampler step behind the two C entry points (dg_sampler_step, dg_sampler_step_noalloc): all
+// arguments are checked first; with clear_ws the workspace is then zeroed on the stream before the
+// launches.  Returns a DG_* status.
+int sampler_step_impl(const void* logits, int logits_dtype, int64_t ld, const int32_t* x_t, int32_t B, int32_t C,
+                      int32_t V, int schedule, const double* t, const double* dt, const float* inv_tau, uint64_t seed,
+                      uint32_t step, int x0_mode, int32_t* x_next, int32_t* x0_hat, int32_t* argmax, float* max_prob,
+                      float* lse, float* entropy, uint8_t* branch, void* workspace, size_t workspace_bytes,
+                      dg_stream_t stream, bool clear_ws);
+
 // Multiprocessor count of the current device (cached per device).
 int num_sms();
 

@@ -11,10 +11,14 @@
 //
 // The array's host-side name is only a stand-in for the symbol, not a device address, so the
 // device address is looked up with cudaGetSymbolAddress, once per device, with that device
-// current, during the first call made on it.  Every call shares the one array: two calls that
-// overlap on the GPU (on different streams, or from different threads) race and corrupt each
-// other's results.  Each call clears the part it uses before launching, so the contents left
-// by an earlier call never matter.
+// current, during the first call made on it; make that first call before any stream capture.
+// The address is cached per device index for the life of the process: a process that calls
+// cudaDeviceReset on a device must not call this entry point on that device afterwards (the
+// reset unloads the module, and the cached address would name memory that is gone).  Every call
+// shares the one array: two calls that overlap on the GPU (on different streams, or from
+// different threads) race and corrupt each other's results.  Each call checks all of its
+// arguments first and only then clears the part of the array it uses and launches, so a refused
+// call enqueues nothing and the contents left by an earlier call never matter.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -78,15 +82,9 @@ extern "C" int dg_sampler_step_noalloc(const void* logits, int logits_dtype, int
         dg::set_error_message(DG_ERR_CUDA, cudaGetErrorString(e));
         return DG_ERR_CUDA;
     }
-    // Counters must start at zero; the previous call may have used the array with another shape.
-    if (need > 0) {
-        e = cudaMemsetAsync(ws, 0, need, reinterpret_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) {
-            dg::set_error_message(DG_ERR_CUDA, cudaGetErrorString(e));
-            return DG_ERR_CUDA;
-        }
-    }
-    return dg_sampler_step(logits, logits_dtype, ld, x_t, B, C, V, schedule, t, dt, inv_tau, seed, step, x0_mode,
-                           x_next, x0_hat, argmax, max_prob, lse, entropy, branch, ws,
-                           static_cast<size_t>(DG_NOALLOC_SCRATCH_BYTES), stream);
+    // Counters must start at zero (the previous call may have used the array with another shape):
+    // cleared on the stream after every argument check has passed.
+    return dg::sampler_step_impl(logits, logits_dtype, ld, x_t, B, C, V, schedule, t, dt, inv_tau, seed, step,
+                                 x0_mode, x_next, x0_hat, argmax, max_prob, lse, entropy, branch, ws,
+                                 static_cast<size_t>(DG_NOALLOC_SCRATCH_BYTES), stream, true);
 }

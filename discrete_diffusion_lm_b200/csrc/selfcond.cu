@@ -95,9 +95,9 @@ struct WaitCtl {
 __device__ __forceinline__ bool aborted(const WaitCtl* c) { return *reinterpret_cast<const volatile int*>(&c->abort) != 0; }
 
 // Wait for the phase with the given parity to complete.  Gives up (returning false) when another
-// thread of the CTA has aborted or after ctl->limit cycles, recording the expiry.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
-    if (mbar_try_wait(bar, parity)) return true;
+// thread of the CTA has aborted or after ctl->limit cycles, recording the expiry.  The first probe
+// is inlined at every call site; only a phase not yet complete pays for the out-of-line loop.
+__device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -108,6 +108,9 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* 
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* ctl) {
+    return mbar_try_wait(bar, parity) || mbar_wait_loop(bar, parity, ctl);
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -478,6 +481,14 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
                  : "memory");
 }
+// One commit that arrives on the barrier at the same shared-memory offset in both CTAs of the pair
+// (own_bar: the executing CTA's shared-memory address of it).
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t own_bar) {
+    const uint16_t mask = 0x3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(own_bar), "h"(mask)
+                 : "memory");
+}
 
 template <bool kBf16, int kNT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
@@ -615,10 +626,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // ---------------------------------------------------------------- MMA issuer (leader)
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(2 * kTileM, G::kMmaN);
-            const uint32_t eempty_own = map_to_rank(smem_u32(&eempty[0]), 0);
-            const uint32_t eempty_peer = map_to_rank(smem_u32(&eempty[0]), 1);
-            const uint32_t lempty_own = map_to_rank(smem_u32(&lempty[0]), 0);
-            const uint32_t lempty_peer = map_to_rank(smem_u32(&lempty[0]), 1);
             for (int i = 0; i < nkb; ++i) {
                 const int es = i % kES, ls = i % kLS;
                 if (!mbar_wait(&efull[es], (i / kES) & 1, wc)) break;
@@ -637,10 +644,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         umma_bf16_pair(tmem + nh * G::kMmaN, adesc, bdesc, idesc, (i > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit_pair(eempty_own + es * 8);
-                umma_commit_pair(eempty_peer + es * 8);
-                umma_commit_pair(lempty_own + ls * 8);
-                umma_commit_pair(lempty_peer + ls * 8);
+                umma_commit_pair_both(smem_u32(&eempty[es]));
+                umma_commit_pair_both(smem_u32(&lempty[ls]));
             }
             umma_commit_pair(map_to_rank(smem_u32(accum), 0));
             umma_commit_pair(map_to_rank(smem_u32(accum), 1));

@@ -191,6 +191,22 @@ def test_binding_rejects_host_and_mistyped_tensors(L):
         dg.dg_adaptive_stop(torch.zeros(16), x_t, x_t.long(), 16, 0.5)
 
 
+def test_noalloc_binding_checks_vectors_before_any_call(L):
+    # the allocation-free step takes the same vector checks as dg_sampler_step: a mistyped or short
+    # canvas, or a caller output buffer that is too short, is refused before the library is called
+    logits = torch.zeros(16, 1024, dtype=torch.bfloat16)
+    x_t = torch.zeros(16, dtype=torch.int32)
+    with pytest.raises(TypeError, match="x_t must be torch.int32"):
+        dg.dg_sampler_step_noalloc(logits, x_t.long(), 16, 0.5, 0.1)
+    with pytest.raises(ValueError, match="x_t has 8 elements, 16 are needed"):
+        dg.dg_sampler_step_noalloc(logits, x_t[:8], 16, 0.5, 0.1)
+    out = {"x_next": torch.zeros(8, dtype=torch.int32)}
+    with pytest.raises(ValueError, match="x_next has 8 elements, 16 are needed"):
+        dg.dg_sampler_step_noalloc(logits, x_t, 16, 0.5, 0.1, out=out)
+    with pytest.raises(TypeError, match="lse must be torch.float32"):
+        dg.dg_sampler_step_noalloc(logits, x_t, 16, 0.5, 0.1, out={"lse": torch.zeros(16, dtype=torch.float64)})
+
+
 def _int_expr(src: str) -> int:
     """Value of a #define body made of integer literals, *, << and parentheses."""
     import ast

@@ -47,12 +47,14 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_requests_beyond_the_fixed_array():
-    # 4096 rows of V = 262144 need 32 MiB of scratch: refused before anything is enqueued
+    # 4096 rows of V = 262144 need 32 MiB of scratch: refused before anything is enqueued.  The
+    # device pointers are NULL, so a call that got past the size check would still stop at the
+    # host-side argument checks and never reach a kernel.
     L = dg.lib()
     t = (ctypes.c_double * 16)(*([0.5] * 16))
     dt = (ctypes.c_double * 16)(*([0.1] * 16))
-    rc = L.dg_sampler_step_noalloc(1 << 20, 1, 262144, 1 << 20, 16, 256, 262144, 1, t, dt, None,
-                                   ctypes.c_uint64(0), ctypes.c_uint32(0), 0, 1 << 20, None, None, None, None,
+    rc = L.dg_sampler_step_noalloc(None, 1, 262144, None, 16, 256, 262144, 1, t, dt, None,
+                                   ctypes.c_uint64(0), ctypes.c_uint32(0), 0, None, None, None, None, None,
                                    None, None, None)
     assert rc == 3
     msg = dg.dg_last_error()
