@@ -242,6 +242,92 @@ int32_t dgo_draw_x0(const float* l, int32_t V, double inv_tau, uint64_t seed, ui
 }
 
 /* ------------------------------------------------------------------------ */
+/* Draw x0_hat ~ p0 = softmax(l') by plain (flat) Gumbel-max over the whole  */
+/* vocabulary: x0_hat = argmax_v l'_v + G_v, one Gumbel variate per id from  */
+/* counter (v>>2, row, step, DOM_GUMBEL_TOKEN), word v&3 -- the same words   */
+/* the two-level draw uses inside its winning chunk.  This is the textbook   */
+/* Gumbel-max definition, with no chunking; the tests compare the two-level  */
+/* draw above with it in distribution at the full vocabulary size.  Ties go  */
+/* to the lowest id.  gap: (best - second best) / max(|best|, 1).            */
+/* ------------------------------------------------------------------------ */
+int32_t dgo_draw_x0_flat(const float* l, int32_t V, double inv_tau, uint64_t seed, uint32_t step,
+                         uint32_t row, double* gap)
+{
+    double best = -INFINITY, second = -INFINITY;
+    int32_t winner = 0;
+    uint32_t w[4];
+    for (int32_t v = 0; v < V; ++v) {
+        if ((v & 3) == 0) philox_word4(seed, (uint32_t)v >> 2, row, step, DOM_GUMBEL_TOKEN, w);
+        double score = (double)l[v] * inv_tau + dgo_gumbel(w[v & 3]);
+        if (score > best) {
+            second = best;
+            best = score;
+            winner = v;
+        } else if (score > second) {
+            second = score;
+        }
+    }
+    *gap = V > 1 ? (best - second) / fmax(fabs(best), 1.0) : INFINITY;
+    return winner;
+}
+
+/* Many draws of one row, one per (seed[k], step[k]) key, for the statistical */
+/* pins: flat != 0 runs dgo_draw_x0_flat per key; otherwise the two-level     */
+/* draw of dgo_draw_x0 with chunk width Q, whose per-chunk log-sum-exps do    */
+/* not depend on the key and are computed once (with the same arithmetic as   */
+/* dgo_draw_x0, so every draw equals that function's).                        */
+void dgo_draw_x0_keys(const float* l, int32_t V, double inv_tau, const uint64_t* seeds,
+                      const uint32_t* steps, int32_t n, uint32_t row, int32_t Q, int32_t flat,
+                      int32_t* out)
+{
+    double gap;
+    if (flat) {
+        for (int32_t k = 0; k < n; ++k)
+            out[k] = dgo_draw_x0_flat(l, V, inv_tau, seeds[k], steps[k], row, &gap);
+        return;
+    }
+    int32_t n_chunks = (V + Q - 1) / Q;
+    double* lse_c = (double*)malloc(sizeof(double) * (size_t)n_chunks);
+    for (int32_t c = 0; c < n_chunks; ++c) {
+        int32_t lo = c * Q, hi = lo + Q < V ? lo + Q : V;
+        double m = -INFINITY;
+        for (int32_t v = lo; v < hi; ++v) {
+            double x = (double)l[v] * inv_tau;
+            if (x > m) m = x;
+        }
+        double S = 0.0;
+        for (int32_t v = lo; v < hi; ++v) S += exp((double)l[v] * inv_tau - m);
+        lse_c[c] = m + log(S);
+    }
+    uint32_t w[4];
+    for (int32_t k = 0; k < n; ++k) {
+        double best1 = -INFINITY;
+        int32_t best_chunk = 0;
+        for (int32_t c = 0; c < n_chunks; ++c) {
+            philox_word4(seeds[k], (uint32_t)c >> 2, row, steps[k], DOM_GUMBEL_CHUNK, w);
+            double score = lse_c[c] + dgo_gumbel(w[c & 3]);
+            if (score > best1) {
+                best1 = score;
+                best_chunk = c;
+            }
+        }
+        int32_t lo = best_chunk * Q, hi = lo + Q < V ? lo + Q : V;
+        double best2 = -INFINITY;
+        int32_t winner = lo;
+        for (int32_t v = lo; v < hi; ++v) {
+            philox_word4(seeds[k], (uint32_t)v >> 2, row, steps[k], DOM_GUMBEL_TOKEN, w);
+            double score = (double)l[v] * inv_tau + dgo_gumbel(w[v & 3]);
+            if (score > best2) {
+                best2 = score;
+                winner = v;
+            }
+        }
+        out[k] = winner;
+    }
+    free(lse_c);
+}
+
+/* ------------------------------------------------------------------------ */
 /* The Step reverse transition [TR-Method, Step equation], read as ancestral */
 /* sampling: x0_hat ~ p0 (above), then the exact posterior of the uniform    */
 /* mixture path                                                              */

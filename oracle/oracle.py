@@ -67,6 +67,9 @@ def _declare(L):
     L.dgo_argmax.restype = _i32
     L.dgo_draw_x0.argtypes = [_p, _i32, _f64, _u64, _u32, _u32, _i32, _p, _p]
     L.dgo_draw_x0.restype = _i32
+    L.dgo_draw_x0_flat.argtypes = [_p, _i32, _f64, _u64, _u32, _u32, _p]
+    L.dgo_draw_x0_flat.restype = _i32
+    L.dgo_draw_x0_keys.argtypes = [_p, _i32, _f64, _p, _p, _i32, _u32, _i32, _i32, _p]
     L.dgo_step.argtypes = [_i32, _i32, _f64, _f64, _i32, _u64, _u32, _u32, _p]
     L.dgo_step.restype = _i32
     L.dgo_step_posterior.argtypes = [_i32, _i32, _f64, _f64, _i32, _p]
@@ -151,6 +154,27 @@ def draw_x0(row, inv_tau: float, seed: int, step: int, row_id: int, chunk: int =
     x = lib().dgo_draw_x0(_ptr(r), r.size, float(inv_tau), seed, step, row_id, chunk,
                           _ptr(g[0:]), _ptr(g[1:]))
     return x, float(g[0]), float(g[1])
+
+
+def draw_x0_flat(row, inv_tau: float, seed: int, step: int, row_id: int):
+    """Plain Gumbel-max over the whole row (no chunking): (x0_hat, gap)."""
+    r = _f32(row)
+    g = np.zeros(1, dtype=np.float64)
+    x = lib().dgo_draw_x0_flat(_ptr(r), r.size, float(inv_tau), seed, step, row_id, _ptr(g))
+    return x, float(g[0])
+
+
+def draw_x0_keys(row, inv_tau: float, seeds, steps, row_id: int, chunk: int = GUMBEL_CHUNK,
+                 flat: bool = False) -> np.ndarray:
+    """One draw of the row per (seeds[k], steps[k]) key: the two-level draw (chunk width
+    `chunk`), or plain Gumbel-max with flat=True."""
+    r = _f32(row)
+    sd = np.ascontiguousarray(seeds, dtype=np.uint64)
+    st = np.ascontiguousarray(steps, dtype=np.uint32)
+    out = np.zeros(sd.size, dtype=np.int32)
+    lib().dgo_draw_x0_keys(_ptr(r), r.size, float(inv_tau), _ptr(sd), _ptr(st), sd.size, row_id, chunk,
+                           1 if flat else 0, _ptr(out))
+    return out
 
 
 def step(x_t: int, x0_hat: int, kappa_t: float, kappa_s: float, V: int, seed: int, step_idx: int,

@@ -314,6 +314,36 @@ def test_forward_noise_marginal_and_layout():
     assert np.all((k >= 0) & (k < K))
 
 
+@pytest.mark.parametrize("V", [1024, 262144])
+def test_forward_noise_marginal_million_draws(V):
+    # The forward path marginal kappa delta(x_t, x0) + (1 - kappa)/V, tested per sequence on 10^6
+    # canvas tokens each at four kappa.  Every token counts: its offset (x_t - x0) mod V is 0 with
+    # probability kappa + (1 - kappa)/V and each other offset with (1 - kappa)/V.  V = 1024: all
+    # V offsets are bins; V = 262144: the zero offset plus 256 equal buckets of the others.
+    n_seq, P, K, C = 4, 8, 2, 500_000
+    rng = np.random.default_rng(14 + V)
+    x0 = rng.integers(0, V, (n_seq, P + K * C)).astype(np.int32)
+    t = [0.2, 0.5, 0.8, 1.0]
+    xt, _ = O.forward_noise(x0, n_seq, P, K, C, V, "cosine", t, 17)
+    assert np.array_equal(xt[:, :P], x0[:, :P])
+    for b in range(n_seq):
+        kap = math.cos(math.pi * t[b] / 2) ** 2
+        off = (xt[b, P:].astype(np.int64) - x0[b, P:]) % V
+        assert off.size == 10 ** 6
+        if V <= 4096:
+            counts = np.bincount(off, minlength=V)
+            probs = np.full(V, (1 - kap) / V)
+            probs[0] += kap
+        else:
+            nb = 256
+            other = off[off > 0]
+            bucket = (other - 1) * nb // (V - 1)
+            counts = np.append((off == 0).sum(), np.bincount(bucket, minlength=nb))
+            sizes = np.bincount((np.arange(1, V) - 1) * nb // (V - 1), minlength=nb)
+            probs = np.append(kap + (1 - kap) / V, sizes * (1 - kap) / V)
+        assert chisq_p(counts, probs) > P_MIN
+
+
 def test_forward_noise_kappa_extremes():
     n_seq, P, K, C, V = 2, 5, 3, 50, 1000
     x0 = np.random.default_rng(11).integers(0, V, (n_seq, P + K * C)).astype(np.int32)
