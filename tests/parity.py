@@ -8,7 +8,8 @@ Tolerances (written here, used by every parity test):
     by less than 1e-5 relative; mismatches must lie on such positions and
     number at most 1e-4 of the positions checked;
   * softmax statistics (lse, max-prob, entropy): |gpu - oracle| <= 1e-3;
-  * z = softmax(l) E in bf16: relative Frobenius error <= 2e-2;
+  * z = softmax(l) E in bf16: relative Frobenius error <= 2e-2, over the rows
+    checked together and on each row alone;
   * canvas cross-entropy: |gpu - oracle| <= 1e-3 + 1e-5 |oracle| per row and
     <= 1e-5 relative (+1e-2 absolute) for the per-sequence sums.
 """
@@ -61,3 +62,10 @@ def rel_fro(a: np.ndarray, b: np.ndarray) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def rel_fro_rows(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Relative Frobenius (Euclidean) error of each row of a against the same row of b."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-300)

@@ -213,3 +213,27 @@ def test_draw_frequencies_on_gpu():
     from scipy.stats import chisquare
     assert counts.sum() >= n - 5  # the -30 background carries < 1e-9 of the mass
     assert chisquare(counts, p / p.sum() * counts.sum()).pvalue > 1e-4
+
+
+def test_draw_frequencies_full_vocab_on_gpu():
+    # the GPU's two-level draw at the real size: 4096 rows holding the same full-vocab row (each row
+    # index keys its own Philox counters, so its draw is independent), 25 steps: 102,400 draws.
+    # Frequencies on the 64 most probable ids plus a tail bucket must match softmax (chi-square).
+    from scipy.special import softmax
+    from scipy.stats import chisquare
+    cfg = W.FULL
+    row = W.make_logits(cfg, DEV, rows=1)[0]
+    n = 4096
+    logits = row.unsqueeze(0).expand(n, -1).contiguous()
+    x_t = torch.zeros(n, dtype=torch.int32, device=DEV)
+    p = softmax(row.double().cpu().numpy())
+    top = np.argsort(-p, kind="stable")[:64]
+    lookup = np.full(cfg.V, 64, dtype=np.int64)
+    lookup[top] = np.arange(64)
+    probs = np.append(p[top], 1.0 - p[top].sum())
+    counts = np.zeros(65, dtype=np.int64)
+    for step in range(25):
+        out = dg_sampler_step(logits, x_t, 256, 0.5, 0.1, seed=77, step=step, schedule="cosine")
+        counts += np.bincount(lookup[out["x0_hat"].cpu().numpy()], minlength=65)
+    assert counts.sum() == 25 * n
+    assert chisquare(counts, probs * counts.sum()).pvalue > 1e-4

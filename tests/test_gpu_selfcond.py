@@ -2,9 +2,11 @@
 (tcgen05 tensor cores) through the C ABI.
 
 Bar: relative Frobenius error <= 2e-2 against the oracle's double-precision z, on every row
-for the tiny workload and on sampled rows (spanning every M tile) for the larger ones.  At
-full size a property that holds for any size is checked on every row as well: with a column
-of ones in E, that column of z is sum_v p_v = 1 (up to bf16 rounding).
+for the tiny workload and on sampled rows (spanning every M tile) for the larger ones; at the
+full sizes the bound holds on each sampled row alone (32 seeded rows of the full-vocab canvas;
+4 seeded rows in each of the 16 batched canvases), not only over the rows pooled.  At full size
+a property that holds for any size is checked on every row as well: with a column of ones in E,
+that column of z is sum_v p_v = 1 (up to bf16 rounding).
 """
 import numpy as np
 import pytest
@@ -13,7 +15,7 @@ import torch
 import discrete_diffusion_lm_b200 as dg
 from discrete_diffusion_lm_b200 import dg_sampler_step, dg_selfcond, workloads as W
 from oracle import oracle as O
-from tests.parity import Z_REL_FRO, host_f32, rel_fro
+from tests.parity import Z_REL_FRO, host_f32, rel_fro, rel_fro_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -21,6 +23,22 @@ DEV = "cuda"
 
 def _z_ref(logits, E, rows, inv_tau_rows=None):
     return O.selfcond_rows(host_f32(logits), host_f32(E), rows, inv_tau_rows)
+
+
+def _z_ref_threaded(logits, E, rows):
+    """The oracle's z on many rows of a full-size workload, one row per task on every host core
+    (about 0.4 s per row; ctypes releases the GIL during each call)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    L, Eh = host_f32(logits), host_f32(E)
+    with ThreadPoolExecutor(max(1, min(32, os.cpu_count() or 1))) as pool:
+        return np.concatenate(list(pool.map(lambda r: O.selfcond_rows(L, Eh, [r]), rows)))
+
+
+def _seeded_rows(cfg, per_canvas, seed):
+    rng = np.random.default_rng(seed)
+    return sorted(int(b * cfg.C + i) for b in range(cfg.B)
+                  for i in rng.choice(cfg.C, size=per_canvas, replace=False))
 
 
 def _device_error_clear():
@@ -76,9 +94,12 @@ def test_full_vocab_sampled_rows_and_mass():
     z = dg_selfcond(logits, E, cfg.C, lse=lse)
     torch.cuda.synchronize()
     assert _device_error_clear() == 0
-    rows = [0, 77, 127, 128, 200, 255]
-    err = rel_fro(z.float().cpu().numpy()[rows], _z_ref(logits, E, rows))
-    assert err <= Z_REL_FRO, err
+    rows = sorted(set(_seeded_rows(cfg, 32, 21)) | {0, 127, 128, 255})
+    ref = _z_ref_threaded(logits, E, rows)
+    got = z.float().cpu().numpy()[rows]
+    per_row = rel_fro_rows(got, ref)
+    assert per_row.max() <= Z_REL_FRO, (per_row.max(), rows[int(per_row.argmax())])
+    assert rel_fro(got, ref) <= Z_REL_FRO
     _ones_column_check(logits, E, cfg.C, lse)
 
 
@@ -89,9 +110,12 @@ def test_batched_sampled_rows_and_mass():
     z = dg_selfcond(logits, E, cfg.C)
     torch.cuda.synchronize()
     assert _device_error_clear() == 0
-    rows = [0, 1000, 2049, 4095]
-    err = rel_fro(z.float().cpu().numpy()[rows], _z_ref(logits, E, rows))
-    assert err <= Z_REL_FRO, err
+    rows = _seeded_rows(cfg, 4, 22)  # every canvas (all 16 row pairs of M tiles)
+    ref = _z_ref_threaded(logits, E, rows)
+    got = z.float().cpu().numpy()[rows]
+    per_row = rel_fro_rows(got, ref)
+    assert per_row.max() <= Z_REL_FRO, (per_row.max(), rows[int(per_row.argmax())])
+    assert rel_fro(got, ref) <= Z_REL_FRO
     _ones_column_check(logits, E, cfg.C, None)
 
 
