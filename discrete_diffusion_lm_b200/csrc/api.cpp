@@ -112,24 +112,25 @@ int32_t n_chunks_of(int32_t V) { return (V + kChunk - 1) / kChunk; }
 int32_t n_groups_of(int32_t V) { return (V + 4 * kChunk - 1) / (4 * kChunk); }
 int32_t groups_per_cta_of(int32_t /*n_groups*/) { return kPassWarps; }
 
-// Logits-pass workspace: per-row counters, sequence tickets (canvas CE), then the chunk records.
+// Logits-pass workspace: the call counter and merge ticket, sequence tickets (canvas CE), then the
+// tagged chunk records.
 struct PassWs {
-    unsigned* row_count;
+    unsigned* epoch;
     uint32_t* seq_ticket;
-    float4* rec;
+    unsigned long long* rec;
 };
 size_t pass_ws_bytes(int32_t R, int32_t V, int32_t n_seq) {
-    return align_up(static_cast<size_t>(R) * 4, 256) + align_up(static_cast<size_t>(n_seq) * 4, 256) +
-           static_cast<size_t>(R) * n_chunks_of(V) * 16;
+    return 256 + align_up(static_cast<size_t>(n_seq) * 4, 256) +
+           static_cast<size_t>(R) * n_chunks_of(V) * kRecWords * 8;
 }
-PassWs carve_pass_ws(void* ws, int32_t R, int32_t n_seq) {
+PassWs carve_pass_ws(void* ws, int32_t /*R*/, int32_t n_seq) {
     char* p = static_cast<char*>(ws);
     PassWs w;
-    w.row_count = reinterpret_cast<unsigned*>(p);
-    p += align_up(static_cast<size_t>(R) * 4, 256);
+    w.epoch = reinterpret_cast<unsigned*>(p);
+    p += 256;
     w.seq_ticket = reinterpret_cast<uint32_t*>(p);
     p += align_up(static_cast<size_t>(n_seq) * 4, 256);
-    w.rec = reinterpret_cast<float4*>(p);
+    w.rec = reinterpret_cast<unsigned long long*>(p);
     return w;
 }
 
@@ -263,7 +264,7 @@ int sampler_step_impl(const void* logits, int logits_dtype, int64_t ld, const in
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_count = w.row_count;
+    p.epoch = w.epoch;
     p.x_t = x_t;
     p.key0 = static_cast<uint32_t>(seed);
     p.key1 = static_cast<uint32_t>(seed >> 32);
@@ -360,7 +361,7 @@ int dg_canvas_ce(const void* logits, int logits_dtype, int64_t ld, const int32_t
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_count = w.row_count;
+    p.epoch = w.epoch;
     p.seq_ticket = w.seq_ticket;
     p.x0 = x0;
     p.canvas_idx = canvas_idx;
@@ -434,7 +435,7 @@ int selfcond_impl(const void* logits, int logits_dtype, int64_t ld, int32_t B, i
         p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
         p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
         p.rec = w.rec;
-        p.row_count = w.row_count;
+        p.epoch = w.epoch;
         p.lse = lse_ws;
         std::memcpy(p.inv_tau, sp.inv_tau, sizeof(float) * B);
         const cudaError_t e = launch_logits_pass(p, kPassStats, logits_dtype == DG_BF16, s);
@@ -605,7 +606,7 @@ int dg_sampler_step_eb(const void* logits, int logits_dtype, int64_t ld, int32_t
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_count = w.row_count;
+    p.epoch = w.epoch;
     p.key0 = static_cast<uint32_t>(seed);
     p.key1 = static_cast<uint32_t>(seed >> 32);
     p.step = step;
@@ -789,7 +790,7 @@ int dg_test_merge_stall(const void* logits, int logits_dtype, int64_t ld, int32_
     p.groups_per_cta = groups_per_cta_of(n_groups_of(V));
     p.segs = (n_groups_of(V) + p.groups_per_cta - 1) / p.groups_per_cta;
     p.rec = w.rec;
-    p.row_count = w.row_count;
+    p.epoch = w.epoch;
     p.lse = lse;
     p.inv_tau[0] = 1.0f;
     p.merge_wait_limit = static_cast<long long>(limit_cycles);

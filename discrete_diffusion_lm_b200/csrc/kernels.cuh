@@ -24,8 +24,8 @@ struct PassParams {
     int32_t n_chunks;        // ceil(V / kChunk)
     int32_t groups_per_cta;  // 4-chunk groups per CTA, a multiple of the warps per CTA
     int32_t segs;            // CTAs per row
-    float4* rec;             // [R, n_chunks] per-chunk (raw max, S, T, -)
-    unsigned* row_count;     // [R] streaming CTAs done per row; zero between calls
+    unsigned long long* rec;  // [R, n_chunks, kRecWords] tagged record words (raw max, S, T), see logits_pass.cu
+    unsigned* epoch;          // [2] call counter (tags the records) and the merge CTAs' ticket
     long long merge_wait_limit;  // cycles a merge waits for its row (0: the library default)
     // sampler
     const int32_t* x_t;
@@ -55,6 +55,7 @@ struct PassParams {
 
 constexpr int kPassThreads = 128;
 constexpr int kPassWarps = kPassThreads / 32;
+constexpr int kRecWords = 3;  // 64-bit words per chunk record (bf16 logits use the first two)
 
 cudaError_t launch_logits_pass(const PassParams& p, int kind, int is_bf16, cudaStream_t s);
 // Test hook: the statistics merge kernel alone, with nothing counting the rows (its waits expire).

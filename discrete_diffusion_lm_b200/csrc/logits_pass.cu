@@ -29,13 +29,59 @@ namespace {
 __device__ int g_pass_error = 0;
 constexpr long long kMergeWaitLimit = 4000000000LL;  // SM cycles, about 2 s
 
-__device__ __forceinline__ void red_release_add(unsigned* addr, unsigned v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* addr) {
+
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* addr) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* addr) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* addr, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+}
+
+// Tag of the current call's records, in [1, 65535] (a zeroed workspace holds tag 0).
+__device__ __forceinline__ unsigned call_tag(const PassParams& p) { return ld_relaxed_u32(p.epoch) % 65535u + 1u; }
+
+// Chunk records are published without a fence: every 64-bit word carries the call's tag beside its
+// value, and an aligned 64-bit store is single-copy atomic, so a reader sees either the previous
+// call's word or this call's.  A release per streaming CTA would keep the CTA's slot for a store
+// round trip and cost about 2 us over the pass.  Layout, kRecWords words per chunk:
+//   bf16 logits: w0 = S << 32 | bf16(m_raw) << 16 | tag,  w1 = tag << 32 | T
+//   fp32 logits: w0 = tag << 32 | m_raw,  w1 = tag << 32 | S,  w2 = tag << 32 | T
+template <bool kBf16>
+__device__ __forceinline__ void put_record(unsigned long long* w, float m_raw, float S, float T, unsigned tag) {
+    if (kBf16) {
+        st_relaxed_u64(w, static_cast<unsigned long long>(__float_as_uint(S)) << 32 |
+                              (__float_as_uint(m_raw) & 0xFFFF0000u) | tag);
+        st_relaxed_u64(w + 1, static_cast<unsigned long long>(tag) << 32 | __float_as_uint(T));
+    } else {
+        const unsigned long long t = static_cast<unsigned long long>(tag) << 32;
+        st_relaxed_u64(w, t | __float_as_uint(m_raw));
+        st_relaxed_u64(w + 1, t | __float_as_uint(S));
+        st_relaxed_u64(w + 2, t | __float_as_uint(T));
+    }
+}
+// Chunk j's record as (m_raw, S, T, -); `ok` is cleared unless every word carries `tag`.
+template <bool kBf16>
+__device__ __forceinline__ float4 get_record(const unsigned long long* rec, int32_t j, unsigned tag, bool& ok) {
+    const unsigned long long* w = rec + static_cast<size_t>(j) * kRecWords;
+    if (kBf16) {
+        const unsigned long long a = ld_relaxed_u64(w), b = ld_relaxed_u64(w + 1);
+        ok &= (static_cast<uint32_t>(a) & 0xFFFFu) == tag && static_cast<uint32_t>(b >> 32) == tag;
+        return make_float4(__uint_as_float(static_cast<uint32_t>(a) & 0xFFFF0000u),
+                           __uint_as_float(static_cast<uint32_t>(a >> 32)), __uint_as_float(static_cast<uint32_t>(b)),
+                           0.f);
+    }
+    const unsigned long long a = ld_relaxed_u64(w), b = ld_relaxed_u64(w + 1), c = ld_relaxed_u64(w + 2);
+    ok &= static_cast<uint32_t>(a >> 32) == tag && static_cast<uint32_t>(b >> 32) == tag &&
+          static_cast<uint32_t>(c >> 32) == tag;
+    return make_float4(__uint_as_float(static_cast<uint32_t>(a)), __uint_as_float(static_cast<uint32_t>(b)),
+                       __uint_as_float(static_cast<uint32_t>(c)), 0.f);
 }
 
 // bf16 -1.0e30 (0xF14A), used twice in a 32-bit word: -inf logits are clamped to it so that the
@@ -252,7 +298,8 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
                                        const void* rowp, MergeShared& sh) {
     const int tid = threadIdx.x;
     const int32_t nch = p.n_chunks;
-    const float4* rec = p.rec + static_cast<size_t>(row) * nch;
+    const unsigned long long* rec = p.rec + static_cast<size_t>(row) * nch * kRecWords;
+    const unsigned tag = call_tag(p);
     const float nbig = neg_big(kBf16);
     const bool sampling = kKind == kPassSampler && p.mode != DG_X0_GREEDY;
 
@@ -275,23 +322,33 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         // pin: computed here, before the wait, not where the scores are formed
         asm volatile("" ::"f"(gum[u][0]), "f"(gum[u][1]), "f"(gum[u][2]), "f"(gum[u][3]));
     }
-    // Wait (bounded) until all p.segs streaming CTAs of the row have counted their records.  Every
-    // streaming CTA has started before this grid launches, so the wait depends on no CTA still to
-    // be placed.
-    if (tid == 0) {
-        const unsigned target = static_cast<unsigned>(p.segs);
-        if (ld_acquire(&p.row_count[row]) < target) {
-            const long long t0 = clock64();
-            const long long limit = p.merge_wait_limit > 0 ? p.merge_wait_limit : kMergeWaitLimit;
-            while (ld_acquire(&p.row_count[row]) < target) {
-                __nanosleep(32);
-                if (clock64() - t0 > limit) {
-                    atomicExch(&g_pass_error, 1);
-                    break;
+    // Wait (bounded) until every record this thread will read carries this call's tag: the quads
+    // q = tid + u T that stay in registers (rows up to 512 chunks) and the ones further out, which
+    // are re-read from L2 in each pass below.  Every streaming CTA has started before this grid
+    // launches, so the wait depends on no CTA still to be placed.
+    float4 r[kRecQuads][4];
+    {
+        const long long limit = p.merge_wait_limit > 0 ? p.merge_wait_limit : kMergeWaitLimit;
+        const long long t0 = clock64();
+        bool ready = false;
+        while (true) {
+            ready = true;
+#pragma unroll
+            for (int u = 0; u < kRecQuads; ++u)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int32_t j = 4 * (tid + u * kPassThreads) + k;
+                    r[u][k] = j < nch ? get_record<kBf16>(rec, j, tag, ready) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
                 }
+            for (int32_t j = 4 * (tid + kRecQuads * kPassThreads); j < nch && ready; j += 4 * kPassThreads)
+                for (int k = 0; k < 4 && j + k < nch; ++k) (void)get_record<kBf16>(rec, j + k, tag, ready);
+            if (ready) break;
+            if (clock64() - t0 > limit) {
+                atomicExch(&g_pass_error, 1);
+                break;
             }
+            __nanosleep(64);
         }
-        p.row_count[row] = 0u;  // ready for the next call (its streaming kernel starts after this grid ends)
     }
     __syncthreads();
 
@@ -312,15 +369,6 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         }
     }
 
-    // Quads q = tid + u T (u < kRecQuads) stay in registers: all records of rows up to 512 chunks.
-    float4 r[kRecQuads][4];
-#pragma unroll
-    for (int u = 0; u < kRecQuads; ++u)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int32_t j = 4 * (tid + u * kPassThreads) + k;
-            r[u][k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
-        }
     // What thread 0 needs at the very end, fetched or computed while the records are in flight:
     // the current token, the canvas's Step thresholds and the Step's Philox words.
     int32_t xt = 0;
@@ -345,10 +393,11 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     // Records beyond those (rows longer than 262144 ids) are re-read from L2 in each pass.
     constexpr int kFar = kRecQuads * kPassThreads;
     auto far_quad = [&](int32_t q, float4 (&f)[4]) {
+        bool ok = true;  // checked above
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int32_t j = 4 * q + k;
-            f[k] = j < nch ? ld_cg_f4(rec + j) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+            f[k] = j < nch ? get_record<kBf16>(rec, j, tag, ok) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
         }
     };
 
@@ -552,7 +601,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 template <bool kBf16, int kKind>
 __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kernel(const __grid_constant__ PassParams p) {
     // The merge kernel, launched as a programmatic dependent, may start once every CTA of this grid
-    // has started; it waits for this grid to finish before reading the chunk records.
+    // has started; each merge waits only for its own row's records.
     if (threadIdx.x == 0) grid_launch_dependents();
     const int32_t row = blockIdx.x / p.segs;
     const int32_t seg = blockIdx.x - row * p.segs;
@@ -561,7 +610,8 @@ __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kern
     const float inv_tau = kKind == kPassCE ? 1.0f : p.inv_tau[canvas];
     constexpr int kElt = kBf16 ? 2 : 4;
     const char* rowp = reinterpret_cast<const char*>(p.logits) + static_cast<size_t>(row) * p.ld * kElt;
-    float4* rec = p.rec + static_cast<size_t>(row) * p.n_chunks;
+    unsigned long long* rec = p.rec + static_cast<size_t>(row) * p.n_chunks * kRecWords;
+    const unsigned tag = call_tag(p);
 
     // Groups of 4 chunks (2048 ids) per warp-iteration; this CTA owns groups [g_begin, g_end).
     const int32_t n_groups = (p.V + 4 * kChunk - 1) / (4 * kChunk);
@@ -576,12 +626,9 @@ __global__ void __launch_bounds__(kPassThreads, kBf16 ? 10 : 4) logits_pass_kern
         else
             cs = group_ragged(rowp, kBf16, lo, p.V, lane, inv_tau);
         const int32_t c = 4 * gi + (lane >> 3);
-        if ((lane & 7) == 0 && c < p.n_chunks) rec[c] = make_float4(cs.m_raw, cs.S, cs.T, 0.f);
+        if ((lane & 7) == 0 && c < p.n_chunks)
+            put_record<kBf16>(rec + static_cast<size_t>(c) * kRecWords, cs.m_raw, cs.S, cs.T, tag);
     }
-    // Count this CTA's records for the row: the barrier orders every warp's record stores before
-    // thread 0's release increment (fire-and-forget), which the row's merge acquires.
-    __syncthreads();
-    if (threadIdx.x == 0) red_release_add(&p.row_count[row], 1u);
 }
 
 // Per-row merge of the chunk records: one CTA per row, launched as a programmatic dependent of the
@@ -597,6 +644,12 @@ __global__ void __launch_bounds__(kPassThreads) merge_kernel(const __grid_consta
     constexpr int kElt = kBf16 ? 2 : 4;
     const char* rowp = reinterpret_cast<const char*>(p.logits) + static_cast<size_t>(row) * p.ld * kElt;
     merge_row<kBf16, kKind>(p, row, canvas, inv_tau, rowp, sh);
+    // The last merge CTA advances the call counter: every CTA of this call has read it by then, and
+    // the next call's kernels start after this grid ends.
+    if (threadIdx.x == 0 && atomicAdd(&p.epoch[1], 1u) == gridDim.x - 1) {
+        p.epoch[1] = 0u;
+        p.epoch[0] += 1u;
+    }
 }
 
 }  // namespace
