@@ -4,22 +4,25 @@
 
 A step is one sampler step of the full-vocabulary workload (one canvas of C = 256 tokens,
 V = 262144, d = 2048, bf16 logits and embeddings, cosine schedule, 12 denoising steps per
-block): the logits pass (softmax statistics, argmax, two-level Gumbel-max draw of x0_hat,
-Step posterior) followed by the self-conditioning contraction z = softmax(L) E.  The metric
-is sampler steps/s (and canvas tokens/s = 256 x steps/s), whole job over N GPUs.
+block), made through the public fused entry point dg_sampler_selfcond_step: the logits pass
+(softmax statistics, argmax, two-level Gumbel-max draw of x0_hat, Step posterior) followed by
+the self-conditioning contraction z = softmax(L) E, which starts while the pass finishes.  The
+metric is sampler steps/s (and canvas tokens/s = 256 x steps/s), whole job over N GPUs.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier + synchronize on
 both sides, on the device with CUDA events, max over ranks.  Each step reads its own logits
 buffer out of a rotation whose total size is well above the 126 MB L2 (inputs larger than
-L2).  The per-step launches are replayed from CUDA graphs captured once.  N > 1 runs
-independent replicas, one per GPU (the path has no data exchange): weak scaling.
+L2).  The K steps are one CUDA graph captured beforehand (a denoising loop as a sampler would
+run it), replayed once.  N > 1 runs independent replicas, one per GPU (the path has no data
+exchange): weak scaling.
 
-Also reported: the dominant kernel's roofline (measured peaks), an end-to-end figure
+Also reported: the dominant kernel's roofline (measured burst peaks), an end-to-end figure
 through the public API with host buffers (host->device logits copy and device->host read
 of x_next and z inside the timed region), the training-side kernels (forward noise and
 canvas cross-entropy on the training workload), the CPU oracle timed on a bounded sample
-(rank 0, N = 1; on one thread, and over row blocks on every host core), SM clocks sampled
-during the timed region, and the number of library kernel launches in the timed region.
+(rank 0, N = 1; on one thread, and over row blocks on every host core) together with its
+comparison against one GPU step on the same inputs (`parity`), SM clocks sampled during the
+timed region, and the number of library kernel launches in the timed region.
 
 --impl reference times the CPU oracle (the plain C reference of the same computation) on a
 bounded sample of the same workload, its rows split over every host core.
@@ -160,6 +163,46 @@ def traffic_from_profiles(kernel_file: str, summary_name: str):
 
 
 # ------------------------------------------------------------------------------ our arm
+def workload_config(world: int, nbuf: int, lbytes: int, cfg=None) -> dict:
+    """The `config` of the JSON line: the same dict on both arms."""
+    if cfg is None:
+        from discrete_diffusion_lm_b200 import workloads as W
+        cfg = W.FULL
+    return {"workload": "full-vocab sampler step: 1 canvas, C=256, V=262144, d=2048, bf16, cosine, 12 steps per "
+                        "block; step = logits pass + self-conditioning contraction (fused entry point)",
+            "B": cfg.B, "C": cfg.C, "V": cfg.V, "d": cfg.d, "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: {nbuf} rotating logits buffers of {lbytes / 1e6:.1f} MB "
+                  f"+ E {cfg.V * cfg.d * 2 / 1e9:.2f} GB"}
+
+
+def rotation(cfg) -> tuple:
+    """Number of identical-content logits buffers cycled so that the step's inputs exceed L2."""
+    lbytes = cfg.R * cfg.V * 2
+    return max(2, math.ceil(3 * L2_BYTES / lbytes) + 1), lbytes
+
+
+def graph_of(fn, ks, stream):
+    """One CUDA graph holding fn(k) for every k in ks, in order."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in ks:
+            fn(k)
+    return g
+
+
+def timed_replay(g, stream) -> float:
+    """Device time (ms) of one replay of g, CUDA events on the launching stream."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    stream.synchronize()
+    return a.elapsed_time(b)
+
+
 def run_ours(args, rank, world, local):
     import torch
     import discrete_diffusion_lm_b200 as dg
@@ -177,124 +220,104 @@ def run_ours(args, rank, world, local):
 
     # inputs resident in HBM: a rotation of identical-content logits buffers (> 3x L2 in total)
     base = W.make_logits(cfg, dev)
-    lbytes = base.numel() * base.element_size()
-    nbuf = max(2, math.ceil(3 * L2_BYTES / lbytes) + 1)
+    nbuf, lbytes = rotation(cfg)
     bufs = [base] + [base.clone() for _ in range(nbuf - 1)]
     E = W.make_embedding(cfg, dev)
-    x_buf = [W.make_canvas(cfg, dev), torch.empty(cfg.R, dtype=torch.int32, device=dev)]
+    x0 = W.make_canvas(cfg, dev)
+    x_buf = [x0.clone(), torch.empty(cfg.R, dtype=torch.int32, device=dev)]
     outs = [{k: torch.empty(cfg.R, dtype=dt, device=dev) for k, dt in
-             (("x_next", torch.int32), ("x0_hat", torch.int32), ("argmax", torch.int32), ("max_prob", torch.float32),
+             (("x0_hat", torch.int32), ("argmax", torch.int32), ("max_prob", torch.float32),
               ("lse", torch.float32), ("entropy", torch.float32), ("branch", torch.uint8))} for _ in range(2)]
     z = torch.empty((cfg.R, cfg.d), dtype=torch.bfloat16, device=dev)
     ws_s = torch.zeros(dg.dg_sampler_step_workspace_size(cfg.R, cfg.V), dtype=torch.uint8, device=dev)
     ws_z = torch.zeros(max(256, dg.dg_selfcond_workspace_size(cfg.R, cfg.V, cfg.d, 1, 1, True)), dtype=torch.uint8,
                        device=dev)
 
-    def k1(k):
+    def step(k):  # one sampler step through the public fused entry point
+        t, dt = cfg.times(k % cfg.steps)
+        o = outs[k % 2]
+        o["x_next"] = x_buf[(k + 1) % 2]
+        dg.dg_sampler_selfcond_step(bufs[k % nbuf], x_buf[k % 2], E, cfg.C, t, dt, schedule=cfg.schedule, seed=0,
+                                    step=k, out=o, z=z, ws=ws_s, ws_z=ws_z, stream=stream)
+
+    def k1(k):  # the logits pass alone
         t, dt = cfg.times(k % cfg.steps)
         o = outs[k % 2]
         o["x_next"] = x_buf[(k + 1) % 2]
         dg.dg_sampler_step(bufs[k % nbuf], x_buf[k % 2], cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=k,
                            out=o, ws=ws_s, stream=stream)
 
-    def k2(k):
+    def k2(k):  # the contraction alone (lse of the last logits pass)
         dg.dg_selfcond(bufs[k % nbuf], E, cfg.C, lse=outs[k % 2]["lse"], z=z, ws=ws_z, stream=stream)
 
-    # one graph per kernel per step of a rotation period (step index and buffer are baked in)
-    period = math.lcm(nbuf, 2 * cfg.steps)
     with torch.cuda.stream(stream):
         for k in range(2):
-            k1(k)
-            k2(k)
+            step(k)
     stream.synchronize()
+    K, Wm = args.steps, args.warmup
+    g_warm = graph_of(step, range(Wm), stream)
     c0 = dg.dg_launch_count()
-    g1, g2 = [], []
-    for k in range(period):
-        a, b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(a, stream=stream):
-            k1(k)
-        with torch.cuda.graph(b, stream=stream):
-            k2(k)
-        g1.append(a)
-        g2.append(b)
-    launches_per_step = (dg.dg_launch_count() - c0) / period
+    g_steps = graph_of(step, range(Wm, Wm + K), stream)
+    launches = dg.dg_launch_count() - c0
+    g_k1 = graph_of(k1, range(Wm, Wm + K), stream)
+    g_k2 = graph_of(k2, range(Wm, Wm + K), stream)
     assert dg.dg_device_error() == 0
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    # warm-up
+    # W untimed warm-up steps, then exactly K steps (one graph of K fused steps), events on the stream
     with torch.cuda.stream(stream):
-        for k in range(args.warmup):
-            g1[k % period].replay()
-            g2[k % period].replay()
+        g_warm.replay()
     stream.synchronize()
-
-    K = args.steps
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
     barrier()
     torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
             ev[0].record(stream)
-            for k in range(K):
-                j = (args.warmup + k) % period
-                g1[j].replay()
-                ev[2 * k + 1].record(stream)
-                g2[j].replay()
-                ev[2 * k + 2].record(stream)
+            g_steps.replay()
+            ev[1].record(stream)
         stream.synchronize()
     torch.cuda.synchronize(dev)
     barrier()
-    total_ms = ev[0].elapsed_time(ev[2 * K])
-    k1_us = [ev[2 * k].elapsed_time(ev[2 * k + 1]) * 1e3 for k in range(K)]
-    k2_us = [ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) * 1e3 for k in range(K)]
+    total_ms = ev[0].elapsed_time(ev[1])
     dev_err = dg.dg_device_error()
-
     total_ms, steps_per_s = whole_job_rate(total_ms, K, world, dev)
 
-    # ---- roofline of the dominant kernel (the contraction) and of the logits pass
-    k1_mean = statistics.mean(k1_us)
-    k2_mean = statistics.mean(k2_us)
+    # ---- the two kernels of the step, each in a graph of K back-to-back launches (same inputs)
+    for g in (g_k1, g_k2):
+        timed_replay(g, stream)  # warm
+    k1_us = timed_replay(g_k1, stream) * 1e3 / K
+    k2_us = timed_replay(g_k2, stream) * 1e3 / K
+
+    # ---- roofline of the dominant kernel (the contraction) against the burst peaks: the timed region
+    # lasts milliseconds.  Slower of the tensor and HBM bounds; the other fraction is reported beside.
     flops_k2 = 2.0 * cfg.R * cfg.V * cfg.d
     bytes_k2 = cfg.V * cfg.d * 2 + cfg.R * cfg.V * 2 + cfg.R * cfg.d * 2 + cfg.R * 4
     bytes_k1 = cfg.R * cfg.V * 2 + cfg.R * 4 + cfg.R * 25
     hbm = peaks["hbm_gbs"]
-    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tc = peaks["bf16_tflops"]
     t_tensor_us = flops_k2 / (tc * 1e12) * 1e6
     t_hbm_us = bytes_k2 / (hbm * 1e9) * 1e6
+    tflops = flops_k2 / (k2_us * 1e-6) / 1e12
+    gbs = bytes_k2 / (k2_us * 1e-6) / 1e9
     if t_tensor_us >= t_hbm_us:
-        achieved = flops_k2 / (k2_mean * 1e-6) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc, "unit": "TFLOP/s",
-                "frac": round(achieved / tc, 4)}
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc, "unit": "TFLOP/s",
+                "frac": round(tflops / tc, 4)}
     else:
-        achieved = bytes_k2 / (k2_mean * 1e-6) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4)}
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4)}
     roof["traffic"] = traffic_from_profiles("selfcond.cu", "selfcond_full_vocab.md")
-    roof["kernel"] = "selfcond (z = softmax(L) E, tcgen05)"
-    roof["peak_source"] = f"{peaks['source']} ({'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} bf16)"
+    roof["kernel"] = "selfcond (z = softmax(L) E, tcgen05), its average over K back-to-back launches"
+    roof["peak_source"] = f"{peaks['source']} (burst: HBM copy and bf16 GEMM peaks)"
     roof["slower_bound_us"] = round(max(t_tensor_us, t_hbm_us), 1)
-    roof["frac_of_slower_bound"] = round(max(t_tensor_us, t_hbm_us) / k2_mean, 4)
-    k1_gbs = bytes_k1 / (k1_mean * 1e-6) / 1e9
+    roof["tensor_frac_burst"] = round(tflops / tc, 4)
+    if "bf16_tflops_sustained" in peaks:
+        roof["tensor_frac_sustained"] = round(tflops / peaks["bf16_tflops_sustained"], 4)
+    k1_gbs = bytes_k1 / (k1_us * 1e-6) / 1e9
 
-    # ---- the logits pass alone: its graphs replayed back to back over the same rotating buffers
-    # (inside the step above, each graph's launch gap is charged to the kernel that follows it)
-    with torch.cuda.stream(stream):
-        for k in range(4):
-            g1[k % period].replay()
-    stream.synchronize()
-    ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ka.record(stream)
-        for k in range(48):
-            g1[k % period].replay()
-        kb.record(stream)
-    stream.synchronize()
-    k1_alone = ka.elapsed_time(kb) * 1e3 / 48
-
-    # ---- training-side kernels on the training workload (forward noise + canvas CE + backward)
+    # ---- training-side kernels, entropy-bounded step, FFW, other workloads
     train = bench_train(dg, W, dev, stream, hbm)
     eb = bench_eb(dg, W, dev, stream, bufs, hbm)
     ffw = bench_ffw(dg, W, dev, stream, peaks)
@@ -303,46 +326,52 @@ def run_ours(args, rank, world, local):
     # ---- end to end through the public API with host buffers
     e2e = bench_e2e(dg, W, cfg, dev, E, args, world, barrier, stream)
 
+    # ---- one more fused step on the first buffer, for the CPU oracle's comparison (outside the timed
+    # region; the oracle runs only in the CPU-baseline leg)
+    probe_step = 3
+    t, dt = cfg.times(probe_step)
+    probe = dg.dg_sampler_selfcond_step(base, x0, E, cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=probe_step,
+                                        stream=stream)
+    stream.synchronize()
+    probe_host = {"step": probe_step, "t": t, "dt": dt, "logits": base, "x_t": x0.cpu().numpy(), "E": E,
+                  "out": {k: v.cpu().numpy() for k, v in probe.items() if k != "z"},
+                  "z": probe["z"].float().cpu().numpy()}
+
     line = {
         "metric": METRIC,
         "value": round(steps_per_s, 2),
         "unit": "steps/s",
         "n_gpus": world,
         "steps": K,
-        "warmup": args.warmup,
+        "warmup": Wm,
         "ms_per_step": round(total_ms / K, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; logits N(0,1.5) + Zipf(1.1) boost on 64 ids per row; E ~ N(0, 0.02))",
-        "config": {"workload": "full-vocab sampler step: 1 canvas, C=256, V=262144, d=2048, bf16, cosine, "
-                               "12 steps per block; step = logits pass + self-conditioning contraction",
-                   "B": cfg.B, "C": cfg.C, "V": cfg.V, "d": cfg.d, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {nbuf} rotating logits buffers of {lbytes / 1e6:.1f} MB "
-                         f"+ E {cfg.V * cfg.d * 2 / 1e9:.2f} GB"},
+        "config": workload_config(world, nbuf, lbytes, cfg),
         "canvas_tokens_per_s": round(steps_per_s * cfg.C, 1),
         "roofline": roof,
         "kernels": {
-            "logits_pass_us": round(k1_mean, 2), "logits_pass_GBps": round(k1_gbs, 1),
+            "timing": "each kernel in a graph of K back-to-back launches on the step's inputs (CUDA events)",
+            "logits_pass_us": round(k1_us, 2), "logits_pass_GBps": round(k1_gbs, 1),
             "logits_pass_frac_hbm": round(k1_gbs / hbm, 4),
-            "logits_pass_alone_us": round(k1_alone, 2),
-            "logits_pass_alone_frac_hbm": round(bytes_k1 / (k1_alone * 1e-6) / 1e9 / hbm, 4),
-            "selfcond_us": round(k2_mean, 2),
-            "selfcond_TFLOPs": round(flops_k2 / (k2_mean * 1e-6) / 1e12, 1),
-            "selfcond_frac_tensor_sustained": round(flops_k2 / (k2_mean * 1e-6) / 1e12 / tc, 4),
-            "selfcond_frac_hbm": round(bytes_k2 / (k2_mean * 1e-6) / 1e9 / hbm, 4),
+            "selfcond_us": round(k2_us, 2),
+            "selfcond_TFLOPs": round(tflops, 1),
+            "selfcond_frac_hbm": round(gbs / hbm, 4),
+            "selfcond_frac_tensor_burst": round(tflops / tc, 4),
             "train": train,
             "entropy_bounded": eb,
             "ffw": ffw,
             "other_workloads": configs,
         },
         "e2e": e2e,
-        "gpu_launches": int(round(launches_per_step * K)),
+        "gpu_launches": int(launches),
         "device_error": dev_err,
         "clocks": clocks.summary(),
     }
-    return line
+    return line, probe_host
 
 
 def bench_train(dg, W, dev, stream, hbm):
@@ -566,11 +595,11 @@ def bench_e2e(dg, W, cfg, dev, E, args, world, barrier, stream):
     def one(k):
         dev_logits.copy_(host_logits, non_blocking=True)
         t, dt = cfg.times(k % cfg.steps)
-        out = dg.dg_sampler_step(dev_logits, x_t, cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=k, stream=stream)
-        z = dg.dg_selfcond(dev_logits, E, cfg.C, lse=out["lse"], stream=stream)
+        out = dg.dg_sampler_selfcond_step(dev_logits, x_t, E, cfg.C, t, dt, schedule=cfg.schedule, seed=0, step=k,
+                                          stream=stream)
         x_t.copy_(out["x_next"])
         host_x.copy_(out["x_next"], non_blocking=True)
-        host_z.copy_(z, non_blocking=True)
+        host_z.copy_(out["z"], non_blocking=True)
 
     with torch.cuda.stream(stream):
         for k in range(3):
@@ -595,30 +624,40 @@ class OracleSample:
     """The CPU oracle (plain C, double precision, as it stands) on a bounded sample of the
     full-vocab workload: the logits-pass work (statistics, argmax, two-level draw, Step) on
     `rows1` rows and the contraction z = softmax(l) E on `rows2` rows over a fraction `vfrac` of
-    the vocabulary; the measured time is scaled to one step (256 rows, all of V)."""
+    the vocabulary; the measured time is scaled to one step (256 rows, all of V).  With `probe`
+    (the GPU's inputs and outputs of one step) the sample runs on exactly those inputs, and the
+    single-thread run's results are compared with the GPU's."""
 
-    def __init__(self, rows1: int, rows2: int, vfrac: int, cfg=None):
+    def __init__(self, rows1: int, rows2: int, vfrac: int, cfg=None, probe=None):
         import numpy as np
         from discrete_diffusion_lm_b200 import workloads as W
         self.cfg = cfg = cfg or W.FULL
         self.rows1, self.rows2, self.vfrac = rows1, rows2, vfrac
+        self.probe = probe
         n = max(rows1, rows2)
-        self.L = W.make_logits(cfg, "cpu", rows=n).float().numpy()
+        if probe is not None:
+            self.L = probe["logits"][:n].float().cpu().numpy()
+            self.E = probe["E"][: cfg.V // vfrac].float().cpu().numpy()
+            self.x_t = np.ascontiguousarray(probe["x_t"][:rows1])
+            self.t, self.dt, self.step = probe["t"], probe["dt"], probe["step"]
+        else:
+            self.L = W.make_logits(cfg, "cpu", rows=n).float().numpy()
+            self.E = W.make_embedding(cfg, "cpu")[: cfg.V // vfrac].float().numpy()
+            self.x_t = np.zeros(rows1, dtype=np.int32)
+            (self.t, self.dt), self.step = cfg.times(0), 0
         self.Vs = cfg.V // vfrac
-        self.E = W.make_embedding(cfg, "cpu")[: self.Vs].float().numpy()
         self.Ls = np.ascontiguousarray(self.L[:rows2, : self.Vs])
-        self.x_t = np.zeros(rows1, dtype=np.int32)
+        self.results = None
 
     def _pass(self, a: int, b: int):
         from oracle import oracle as O
         cfg = self.cfg
-        t, dt = cfg.times(0)
-        O.sampler_step(self.L[a:b], self.x_t[a:b], 1, b - a, cfg.V, cfg.schedule, t[:1], dt[:1], None, 0, 0,
-                       "sample")
+        return O.sampler_step(self.L[a:b], self.x_t[a:b], 1, b - a, cfg.V, cfg.schedule, self.t[:1], self.dt[:1], None,
+                              0, self.step, "sample")
 
     def _z(self, a: int, b: int):
         from oracle import oracle as O
-        O.selfcond_rows(self.Ls, self.E, list(range(a, b)))
+        return O.selfcond_rows(self.Ls, self.E, list(range(a, b)))
 
     def _what(self) -> str:
         c = self.cfg
@@ -631,10 +670,11 @@ class OracleSample:
         """Single thread: the logits pass on all `rows1` rows, z on the first `rows2` rows."""
         rows2 = rows2 or self.rows2
         t0 = time.perf_counter()
-        self._pass(0, self.rows1)
+        ref = self._pass(0, self.rows1)
         t1 = time.perf_counter()
-        self._z(0, rows2)
+        zr = self._z(0, rows2)
         t2 = time.perf_counter()
+        self.results = (ref, zr)
         step_s = self._per_step(t1 - t0, self.rows1, t2 - t1, rows2)
         return {"value": 1.0 / step_s, "unit": "steps/s", "cores": 1, "kind": "oracle", "cpu_seconds": t2 - t0,
                 "sample": f"{self._what()}: logits pass on {self.rows1} rows + z on {rows2} rows over "
@@ -665,6 +705,31 @@ class OracleSample:
                           f"1/{self.vfrac} of V, split into row blocks over {threads} threads, scaled to "
                           f"{self.cfg.R} rows x full V per step"}
 
+    def parity(self, near_tie_rel: float = 1e-5) -> dict:
+        """The single-thread run's results against the GPU's outputs of the same step (the probe):
+        integer outputs compared exactly, sampled tokens exactly except at near-ties (top-two
+        Gumbel-perturbed scores within near_tie_rel relative), statistics by their largest absolute
+        difference, z by its relative Frobenius error per row."""
+        import numpy as np
+        ref, zr = self.results
+        g = self.probe["out"]
+        n = self.rows1
+        near = (ref["gap1"] < near_tie_rel) | (ref["gap2"] < near_tie_rel)
+        bad = g["x0_hat"][:n] != ref["x0_hat"]
+        same = ~bad
+        zg = self.probe["z"][: zr.shape[0]].astype(np.float64)
+        zrow = np.linalg.norm(zg - zr, axis=1) / np.maximum(np.linalg.norm(zr, axis=1), 1e-300)
+        return {"rows": int(n), "argmax_mismatches": int((g["argmax"][:n] != ref["argmax"]).sum()),
+                "near_ties": int(near.sum()), "x0_hat_mismatches": int(bad.sum()),
+                "x0_hat_mismatches_off_near_ties": int((bad & ~near).sum()),
+                "x_next_mismatches_where_x0_hat_agrees": int((g["x_next"][:n][same] != ref["x_next"][same]).sum()),
+                "max_stat_abs_err": float(max(np.abs(g[k][:n].astype(np.float64) - ref[k]).max()
+                                              for k in ("lse", "max_prob", "entropy"))),
+                "z_rows": int(zr.shape[0]), "z_rel_fro_max_row": float(zrow.max()),
+                "z_rel_fro": float(np.linalg.norm(zg - zr) / np.linalg.norm(zr)),
+                "source": f"CPU-baseline leg: the oracle on the bench's own logits buffer and canvas, step "
+                          f"{self.probe['step']}, against one fused GPU step on the same inputs"}
+
 
 def host_cores(cpu_max_path: str = "/sys/fs/cgroup/cpu.max") -> int:
     """Cores this process may run on: its affinity mask, capped by a cgroup CPU quota if any."""
@@ -681,18 +746,20 @@ def host_cores(cpu_max_path: str = "/sys/fs/cgroup/cpu.max") -> int:
     return n
 
 
-def oracle_baseline() -> tuple:
+def oracle_baseline(probe=None) -> tuple:
     """About 10-20 s of single-threaded oracle work on rank 0, then the same routines on every
-    host core (z on up to three rows per thread, at most all 256)."""
+    host core (z on up to three rows per thread, at most all 256).  With the GPU's probe step, the
+    single-thread run is also compared with the GPU's outputs (the `parity` object)."""
     cores = host_cores()
     single_rows2 = 24
-    samp = OracleSample(rows1=256, rows2=min(256, max(single_rows2, 3 * cores)), vfrac=1)
+    samp = OracleSample(rows1=256, rows2=min(256, max(single_rows2, 3 * cores)), vfrac=1, probe=probe)
     one = samp.run(rows2=single_rows2)
+    par = samp.parity() if probe is not None else None
     many = samp.run_threads(cores)
     for r in (one, many):
         r["value"] = round(r["value"], 6)
         r["cpu_seconds"] = round(r["cpu_seconds"], 1)
-    return one, many
+    return one, many, par
 
 
 def run_reference(args, rank, world):
@@ -708,12 +775,11 @@ def run_reference(args, rank, world):
     secs = sum(1.0 / r["value"] for r in res)  # extrapolated seconds for K full steps
     v = args.steps / secs
     cfg = samp.cfg
+    nbuf, lbytes = rotation(cfg)
     return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / v, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": "full-vocab sampler step: 1 canvas, C=256, V=262144, d=2048, bf16, cosine, "
-                                   "12 steps per block; step = logits pass + self-conditioning contraction",
-                       "B": cfg.B, "C": cfg.C, "V": cfg.V, "d": cfg.d},
+            "config": workload_config(world, nbuf, lbytes, cfg),
             "cpu_baseline": {"value": round(v, 6), "unit": "steps/s", "cores": cores, "kind": "oracle",
                              "sample": res[0]["sample"]},
             "e2e": {"value": round(v, 6), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -740,9 +806,9 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
                                              timeout=__import__("datetime").timedelta(seconds=120))
-    line = run_ours(args, rank, world, local)
+    line, probe = run_ours(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"], line["cpu_baseline_all_cores"] = oracle_baseline()
+        line["cpu_baseline"], line["cpu_baseline_all_cores"], line["parity"] = oracle_baseline(probe)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

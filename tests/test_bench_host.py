@@ -76,6 +76,44 @@ def test_reference_arm_prints_one_json_line():
     assert rec["impl"] == "reference" and rec["unit"] == "steps/s" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["value"] == rec["value"]
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["warmup"] >= 3
+    # the same config dict as the GPU arm's line (same workload, layout and rotation)
+    nbuf, lbytes = bench.rotation(bench_cfg())
+    assert rec["config"] == bench.workload_config(1, nbuf, lbytes)
+
+
+def bench_cfg():
+    from discrete_diffusion_lm_b200 import workloads as W
+    return W.FULL
+
+
+def test_parity_leg_compares_the_oracle_with_a_probe_step():
+    # the CPU-baseline leg's comparison, fed a probe whose "GPU" outputs are the oracle's own on the
+    # same inputs: nothing differs; a planted wrong token (in a copy of the outputs) is counted
+    import numpy as np
+    import torch
+    from discrete_diffusion_lm_b200 import workloads as W
+    from oracle import oracle as O
+    cfg = W.TINY
+    L = W.make_logits(cfg, "cpu")
+    E = W.make_embedding(cfg, "cpu")
+    x_t = W.make_canvas(cfg, "cpu").numpy()
+    t, dt = cfg.times(3)
+    ref = O.sampler_step(L.numpy(), x_t, 1, cfg.R, cfg.V, cfg.schedule, t[:1], dt[:1], None, 0, 3, "sample")
+    zr = O.selfcond_rows(L.numpy(), E.numpy(), list(range(cfg.R)))
+    probe = {"step": 3, "t": t, "dt": dt, "logits": L, "x_t": x_t, "E": E,
+             "out": {k: np.asarray(ref[k]).astype(np.float32 if k in ("lse", "max_prob", "entropy") else np.int32)
+                     for k in ("x_next", "x0_hat", "argmax", "lse", "max_prob", "entropy")},
+             "z": zr.astype(np.float32)}
+    samp = bench.OracleSample(rows1=cfg.R, rows2=4, vfrac=1, cfg=cfg, probe=probe)
+    samp.run(rows2=4)
+    par = samp.parity()
+    assert par["rows"] == cfg.R and par["argmax_mismatches"] == 0 and par["x0_hat_mismatches"] == 0
+    assert par["x_next_mismatches_where_x0_hat_agrees"] == 0 and par["max_stat_abs_err"] < 1e-6
+    assert par["z_rows"] == 4 and par["z_rel_fro_max_row"] < 1e-6
+    probe["out"]["argmax"] = probe["out"]["argmax"].copy()
+    probe["out"]["argmax"][5] += 1
+    assert samp.parity()["argmax_mismatches"] == 1
+    assert torch.is_tensor(L)
 
 
 def test_host_cores_honours_a_cgroup_quota(tmp_path):
