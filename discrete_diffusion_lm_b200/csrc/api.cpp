@@ -10,6 +10,7 @@
 #include <string>
 
 #include "../../include/dg.h"
+#include "../../include/dg_test.h"
 #include "kernels.cuh"
 
 namespace dg {

@@ -25,9 +25,11 @@
  *     A workspace must be zero-filled before its first use, and again before
  *     it is reused for a call of a different shape (rows, V, n_seq): the
  *     layout inside it depends on the shape.  Every call that returns DG_OK
- *     leaves the counters inside it at zero, so one workspace serves any
- *     number of successive same-shape calls on one stream.  Two calls that
- *     run at the same time need two workspaces.
+ *     leaves it ready for the next call of the same shape (its counters back
+ *     at zero, the call counter that tags the logits pass's records
+ *     advanced), so one workspace serves any number of successive same-shape
+ *     calls on one stream.  Two calls that run at the same time need two
+ *     workspaces.
  *   - Per-canvas scalars (t, dt, inv_tau) are HOST arrays, read during the
  *     call; everything else named "device" is device memory.
  *   - All work is enqueued asynchronously on `stream` (a cudaStream_t;
@@ -304,46 +306,14 @@ int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed
 /* [d_ff, d]; hidden: device bf16 [rows, d_ff] (caller-owned scratch, also  */
 /* an output); z_out: device bf16 [rows, d]; all row-major, 16-byte aligned */
 /* and not aliased.  d, d_ff multiples of 64 in [64, 16384].  Workspace     */
-/* (256-byte aligned, no zeroing needed): dg_ffw_workspace_size bytes (may  */
-/* be 0).  Two contraction launches (+ their split sums) on `stream`.      */
+/* (256-byte aligned, zeroed before first use: it holds the split-K        */
+/* counters): dg_ffw_workspace_size bytes (may be 0).  Two contraction     */
+/* launches on `stream`.                                                    */
 /* ------------------------------------------------------------------------ */
 size_t dg_ffw_workspace_size(int32_t rows, int32_t d, int32_t d_ff);
 
 int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* W1, const void* W2,
            void* hidden, void* z_out, void* workspace, size_t workspace_bytes, dg_stream_t stream);
-
-/* ------------------------------------------------------------------------ */
-/* Failure-detection test hooks (the pages have no counterpart).  Every wait */
-/* inside the library's kernels is bounded; these entry points make a wait  */
-/* run out on purpose -- without any fault, trap or endless loop -- so that */
-/* tests can check that the kernel gives up, reports through                */
-/* dg_device_error() (code 1) and leaves the device usable.                 */
-/* dg_test_bounded_wait: one thread waits on a barrier nothing arrives on;  */
-/*   the wait gives up after limit_cycles (> 0) SM clock cycles.             */
-/* dg_test_selfcond_stall: dg_selfcond with the copy of one 64-id block of  */
-/*   E never issued (stalled_block >= 0, in [0, ceil(V/64)) to take effect) */
-/*   and every wait limited to limit_cycles: the CTAs that need the block   */
-/*   abort, drain their in-flight copies, free their tensor memory and      */
-/*   return.  z is then incomplete.  Same arguments as dg_selfcond otherwise.*/
-/* ------------------------------------------------------------------------ */
-int dg_test_bounded_wait(uint32_t limit_cycles, dg_stream_t stream);
-
-/* dg_test_merge_stall: the logits pass's per-row merge kernel alone (the   */
-/*   statistics epilogue), with nothing counting its rows: every row's wait */
-/*   gives up after limit_cycles (> 0), records device error 1, and the     */
-/*   merge finishes on whatever the workspace holds (lse is then            */
-/*   meaningless).  logits as dg_sampler_step with B = 1, C = rows; lse:    */
-/*   device float [rows]; workspace: dg_sampler_step_workspace_size(rows, V)*/
-/*   bytes, zeroed.                                                         */
-int dg_test_merge_stall(const void* logits, int logits_dtype, int64_t ld, int32_t rows, int32_t V,
-                        float* lse, void* workspace, size_t workspace_bytes, uint32_t limit_cycles,
-                        dg_stream_t stream);
-
-int dg_test_selfcond_stall(const void* logits, int logits_dtype, int64_t ld, int32_t B, int32_t C,
-                           int32_t V, const float* inv_tau, const float* lse, const void* E,
-                           int embed_dtype, int32_t d, void* z, void* workspace,
-                           size_t workspace_bytes, dg_stream_t stream, int32_t stalled_block,
-                           uint32_t limit_cycles);
 
 /* ------------------------------------------------------------------------ */
 /* Allocation-free sampler step.  The pages have no counterpart: this entry  */

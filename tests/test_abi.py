@@ -1,6 +1,7 @@
 """CPU checks of the C ABI: the library builds for sm_100a, loads, exports every function
-include/dg.h declares, and rejects bad arguments with a status and a message before any
-launch (these calls never reach a device, so they are safe with or without a GPU)."""
+include/*.h declares (dg.h, the sampler's interface, and dg_test.h, its failure-detection test
+hooks), and rejects bad arguments with a status and a message before any launch (these calls
+never reach a device, so they are safe with or without a GPU)."""
 import ctypes
 import os
 import re
@@ -13,6 +14,7 @@ from discrete_diffusion_lm_b200 import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "dg.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include"))) if h.endswith(".h")]
 
 FAKE = 1 << 20  # an aligned non-null address that is never dereferenced (calls fail validation first)
 
@@ -23,17 +25,22 @@ def L():
     return dg.lib()
 
 
-def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", text)))
+def declared_functions(path=None):
+    names = set()
+    for h in ([path] if path else HEADERS):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
     names = declared_functions()
     assert {"dg_sampler_step", "dg_selfcond", "dg_forward_noise", "dg_canvas_ce"} <= set(names)
+    assert {"dg_test_bounded_wait", "dg_test_merge_stall", "dg_test_selfcond_stall"} <= set(names)
     for n in names:
-        assert hasattr(L, n), f"{n} declared in dg.h but not exported"
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    # the sampler's interface header declares no test hook
+    assert not [n for n in declared_functions(HEADER) if n.startswith("dg_test_")]
 
 
 def test_version_and_launch_count(L):
