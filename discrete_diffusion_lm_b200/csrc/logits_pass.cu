@@ -270,13 +270,68 @@ __device__ __forceinline__ void unpack_quad(const RawQuad& q, int32_t v, int32_t
 
 // Level-1 Gumbel score of a chunk: its log-sum-exp of l' plus its Gumbel variate (-inf for a chunk
 // without mass).
+// ln S with the hardware logarithm: S >= 1 for a chunk with mass (its maximum contributes 1), so the
+// absolute error stays near 1e-6, far inside the near-tie allowance of the scores (1e-5 relative).
 __device__ __forceinline__ float chunk_score(float m_raw, float S, float inv_tau, float gumbel) {
-    return (m_raw * inv_tau + logf(S)) + gumbel;
+    return (m_raw * inv_tau + __logf(S)) + gumbel;
+}
+
+// Running statistics of a set of chunk records: the first chunk holding the raw maximum, the level-1
+// winner (score, chunk), and S, T of the chunks with mass relative to the reference `ref`
+// (S = sum exp(l' - ref), T = sum exp(l' - ref)(l' - ref)).
+struct RowAcc {
+    float mv, bs, ref, S, T;
+    int jm, bj;
+};
+__device__ __forceinline__ void acc_init(RowAcc& a) {
+    a.mv = a.bs = a.ref = -INFINITY;
+    a.S = a.T = 0.f;
+    a.jm = a.bj = 0x7fffffff;
+}
+// (S, T) of b folded into a: both rescaled to the larger reference.
+__device__ __forceinline__ void acc_sums(RowAcc& a, float ref, float S, float T) {
+    if (!(S > 0.f)) return;
+    if (!(a.S > 0.f)) {
+        a.ref = ref;
+        a.S = S;
+        a.T = T;
+        return;
+    }
+    const float nr = fmaxf(a.ref, ref);
+    const float da = a.ref - nr, db = ref - nr;
+    const float ea = __expf(da), eb = __expf(db);
+    a.T = fmaf(ea, fmaf(a.S, da, a.T), eb * fmaf(S, db, T));
+    a.S = fmaf(a.S, ea, S * eb);
+    a.ref = nr;
+}
+// b folded into a (both sets' statistics): larger value wins, equal values go to the smaller chunk.
+__device__ __forceinline__ void acc_merge(RowAcc& a, const RowAcc& b) {
+    if (b.mv > a.mv || (b.mv == a.mv && b.jm < a.jm)) {
+        a.mv = b.mv;
+        a.jm = b.jm;
+    }
+    if (b.bs > a.bs || (b.bs == a.bs && b.bj < a.bj)) {
+        a.bs = b.bs;
+        a.bj = b.bj;
+    }
+    acc_sums(a, b.ref, b.S, b.T);
+}
+__device__ __forceinline__ RowAcc acc_shfl_xor(const RowAcc& a, int o) {
+    RowAcc b;
+    b.mv = __shfl_xor_sync(0xffffffffu, a.mv, o);
+    b.bs = __shfl_xor_sync(0xffffffffu, a.bs, o);
+    b.ref = __shfl_xor_sync(0xffffffffu, a.ref, o);
+    b.S = __shfl_xor_sync(0xffffffffu, a.S, o);
+    b.T = __shfl_xor_sync(0xffffffffu, a.T, o);
+    b.jm = __shfl_xor_sync(0xffffffffu, a.jm, o);
+    b.bj = __shfl_xor_sync(0xffffffffu, a.bj, o);
+    return b;
 }
 
 struct MergeShared {
     float f[2 * kPassWarps];
     int i[2 * kPassWarps];
+    RowAcc acc[kPassWarps];
     int flag;
 };
 
@@ -285,9 +340,9 @@ struct MergeShared {
 // registers, so one Philox call serves four chunk Gumbel variates), then the two chunks that must
 // be re-read (the one holding the argmax and the level-1 winner), fetched together.
 //
-// Three block-wide exchanges: (1) the argmax over the chunk maxima and the level-1 winner, which
-// fixes both chunks to re-read, so their loads are in flight during (2) the log-sum-exp merge of
-// (S, T); (3) the argmax inside the argmax chunk and the level-2 winner.
+// Two block-wide exchanges: (1) the argmax over the chunk maxima, the level-1 winner and the
+// log-sum-exp merge of (S, T) together (an online merge at a running reference), which fixes both
+// chunks to re-read; (2) the argmax inside the argmax chunk and the level-2 winner.
 // A re-read chunk is kQuads quads of four consecutive ids per thread: ids lo + 4 (tid + u T) + k.
 constexpr int kQuads = kChunk / (4 * kPassThreads);
 constexpr int kRecQuads = (512 / 4 + kPassThreads - 1) / kPassThreads;
@@ -401,34 +456,31 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         }
     };
 
-    // (1) The first chunk holding the row maximum of the raw chunk maxima, and the level-1 winner
-    // of the chunk scores lse_c + G_c.
-    float mv = -INFINITY, bs = -INFINITY;
-    int jm = 0x7fffffff, bj = 0x7fffffff;
-    auto scan_quad = [&](int32_t q, const float4 (&f)[4], const float (&g)[4]) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            if (f[k].x > mv) {  // ascending ids, strict: the first maximum wins
-                mv = f[k].x;
-                jm = 4 * q + k;
-            }
+    // (1) One block exchange for all of the row's statistics: each thread folds its records (the
+    // first chunk holding the raw maximum, the level-1 winner of the chunk scores lse_c + G_c, and
+    // (S, T) at a running reference), then the warps fold theirs by shuffles in a fixed tree and
+    // every thread folds the warps' results in warp order (deterministic).
+    RowAcc acc;
+    acc_init(acc);
+    auto fold = [&](int32_t j, const float4& f, float g) {
+        if (j >= nch) return;
+        if (f.x > acc.mv) {  // ascending chunks within a thread, strict: the first maximum wins
+            acc.mv = f.x;
+            acc.jm = j;
+        }
         if (sampling) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int32_t j = 4 * q + k;
-                if (j < nch) {
-                    const float sc = chunk_score(f[k].x, f[k].y, inv_tau, g[k]);
-                    if (sc > bs) {
-                        bs = sc;
-                        bj = j;
-                    }
-                }
+            const float sc = chunk_score(f.x, f.y, inv_tau, g);
+            if (sc > acc.bs) {
+                acc.bs = sc;
+                acc.bj = j;
             }
         }
+        acc_sums(acc, f.x * inv_tau, f.y, f.z);
     };
 #pragma unroll
     for (int u = 0; u < kRecQuads; ++u)
-        if (4 * (tid + u * kPassThreads) < nch) scan_quad(tid + u * kPassThreads, r[u], gum[u]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) fold(4 * (tid + u * kPassThreads) + k, r[u][k], gum[u][k]);
     for (int32_t q = tid + kFar; 4 * q < nch; q += kPassThreads) {
         float4 f[4];
         far_quad(q, f);
@@ -440,19 +492,37 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 #pragma unroll
             for (int k = 0; k < 4; ++k) g[k] = gumbel_from_word(word_of(w, k));
         }
-        scan_quad(q, f, g);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) fold(4 * q + k, f[k], g[k]);
     }
-    block_argmax2<kPassWarps>(mv, jm, bs, bj, sh.f, sh.i);
-    const float m_raw = mv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc_merge(acc, acc_shfl_xor(acc, o));
+    if ((tid & 31) == 0) sh.acc[tid >> 5] = acc;
+    __syncthreads();
+    acc = sh.acc[0];
+#pragma unroll
+    for (int w = 1; w < kPassWarps; ++w) acc_merge(acc, sh.acc[w]);
+
+    const float m_raw = acc.mv;
+    int32_t jm = acc.jm, bj = acc.bj;
     if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
     if (!sampling || bj >= nch) bj = jm;  // greedy, or NaN scores only
     const float m_row = m_raw * inv_tau;
+    // (S, T) at the row maximum (the reference is the maximum unless the maximum chunk is masked)
+    float S = acc.S, T = acc.T;
+    if (S > 0.f && acc.ref != m_row) {
+        const float d = acc.ref - m_row;
+        const float e = __expf(d);
+        T = e * fmaf(S, d, T);
+        S *= e;
+    }
 
     // Both re-read chunks are known: quads of ids lo + 4 (tid + u T) .. + 3 of each, loaded now as
-    // raw words and used only after the next exchange, so the loads overlap it.
+    // raw words, with the level-2 chunk's Philox words computed while the loads are in flight.
     const int32_t alo = jm * kChunk, ahi = min(alo + kChunk, p.V);
     const int32_t glo = bj * kChunk, ghi = min(glo + kChunk, p.V);
     RawQuad araw[kQuads], graw[kQuads];
+    uint4 tw[kQuads];
     if (kKind == kPassSampler) {
 #pragma unroll
         for (int u = 0; u < kQuads; ++u) {
@@ -460,29 +530,15 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
             araw[u] = load_quad<kBf16>(rowp, alo + o, ahi);
             graw[u] = load_quad<kBf16>(rowp, glo + o, ghi);
         }
+#pragma unroll
+        for (int u = 0; u < kQuads; ++u) {
+            const int32_t vg0 = glo + 4 * (tid + u * kPassThreads);
+            tw[u] = sampling ? philox4x32_10(make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row),
+                                                        p.step, kDomTokenGumbel),
+                                             p.key0, p.key1)
+                             : make_uint4(0u, 0u, 0u, 0u);
+        }
     }
-
-    // (2) Log-sum-exp merge of (S, T) relative to the row maximum.
-    float s = 0.f, t = 0.f;
-    auto acc_st = [&](const float4& c) {
-        if (c.x == -INFINITY) return;  // missing chunk
-        const float dm = c.x * inv_tau - m_row;
-        const float f = expf(dm);
-        s = fmaf(c.y, f, s);
-        t = fmaf(f, fmaf(c.y, dm, c.z), t);
-    };
-#pragma unroll
-    for (int u = 0; u < kRecQuads; ++u)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc_st(r[u][k]);
-    for (int32_t q = tid + kFar; 4 * q < nch; q += kPassThreads) {
-        float4 f[4];
-        far_quad(q, f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc_st(f[k]);
-    }
-    block_sum2<kPassWarps>(s, t, sh.f);
-    const float S = s, T = t;
     const float ln_s = logf(S);
     const float lse = m_row + ln_s;
 
@@ -519,7 +575,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     }
 
     // ---- sampler epilogue
-    // (3) The first id of the argmax chunk holding the row maximum, and the level-2 winner
+    // (2) The first id of the argmax chunk holding the row maximum, and the level-2 winner
     // argmax of l'_v + G_v over the level-1 chunk (four ids per Philox call).
     float av[kQuads][4], gv[kQuads][4];
 #pragma unroll
@@ -544,9 +600,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     for (int u = 0; u < kQuads; ++u) {
         const int32_t vg0 = glo + 4 * (tid + u * kPassThreads);
         if (sampling && vg0 < ghi) {
-            const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(vg0) >> 2, static_cast<uint32_t>(row), p.step, kDomTokenGumbel),
-                p.key0, p.key1);
+            const uint4 w = tw[u];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 if (vg0 + k < ghi) {
