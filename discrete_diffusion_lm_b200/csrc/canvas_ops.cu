@@ -10,7 +10,9 @@
 //   zero for the other half.
 //
 // canvas_decide_kernel: one CTA of kDecideThreads threads per canvas (C <= DG_MAX_CANVAS_ROWS), the
-//   decisions of canvas_decide.cuh.
+//   decisions of canvas_decide.cuh.  Launched as a programmatic dependent of the preceding kernel:
+//   its CTAs may be placed while the logits pass's merge runs, and wait (griddepcontrol.wait) for
+//   that grid's completion and its memory before reading any input.
 // ce_backward_kernel: rows along grid y, 16-byte bf16 vectors of a row along grid x, in place.
 // selfcond_drop_kernel: sequences along grid y; a fair Philox coin per sequence decides, dropped
 //   rows are zeroed.
@@ -28,6 +30,7 @@ constexpr int kDecideThreads = 256;
 
 __global__ void __launch_bounds__(kDecideThreads) canvas_decide_kernel(const __grid_constant__ DecideParams p) {
     __shared__ DecideShared sh;
+    grid_dependency_wait();
     decide_canvas<kDecideThreads>(p, blockIdx.x, sh);
 }
 
@@ -99,7 +102,17 @@ __global__ void __launch_bounds__(256) selfcond_drop_kernel(uint16_t* z, int64_t
 
 cudaError_t launch_canvas_decide(const DecideParams& p, int32_t B, cudaStream_t s) {
     if (B < 1 || p.C < 1 || p.C > DG_MAX_CANVAS_ROWS) return cudaErrorInvalidValue;
-    canvas_decide_kernel<<<B, kDecideThreads, 0, s>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B));
+    cfg.blockDim = dim3(kDecideThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, canvas_decide_kernel, p);
+    if (e != cudaSuccess) return e;
     note_launches(1);
     return cudaGetLastError();
 }

@@ -44,7 +44,7 @@ def _entropies(kind, n, rng):
 
 
 @pytest.mark.parametrize("kind", ["uniform", "tied", "tiny", "special"])
-@pytest.mark.parametrize("B,C", [(4, 256), (1, 1), (3, 100), (2, 1024)])
+@pytest.mark.parametrize("B,C", [(4, 256), (1, 1), (3, 100), (2, 1024), (1, 993)])
 @pytest.mark.parametrize("eps", [0.0, 0.3, 7.5, 1e9])
 def test_entropy_accept_matches_oracle(kind, B, C, eps):
     rng = np.random.default_rng(zlib.crc32(f"{kind}-{B}-{C}".encode()))
@@ -59,7 +59,7 @@ def test_entropy_accept_matches_oracle(kind, B, C, eps):
     np.testing.assert_array_equal(out["x_next"].cpu().numpy(), x_ref)
 
 
-@pytest.mark.parametrize("B,C", [(8, 256), (1, 1), (3, 77), (2, 1024)])
+@pytest.mark.parametrize("B,C", [(8, 256), (1, 1), (3, 77), (2, 1024), (5, 33)])
 def test_adaptive_stop_matches_oracle(B, C):
     rng = np.random.default_rng(C)
     H = rng.uniform(0.0, 1.0, B * C).astype(np.float32)
