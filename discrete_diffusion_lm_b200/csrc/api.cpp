@@ -738,6 +738,9 @@ int dg_ffw(const void* z_in, int32_t rows, int32_t d, int32_t d_ff, const void* 
         sp.plain_a = 1;
         sp.act = layer == 0 ? 1 : 0;
         sp.inv_tau[0] = 1.0f;
+        // the second layer may be placed while the first drains: its weight copies start at once,
+        // its hidden-layer copies wait for the preceding grid
+        sp.dependent = layer == 1 ? 1 : 0;
         const cudaError_t e = launch_selfcond(sp, s);
         if (e != cudaSuccess) return cuda_fail(e, layer == 0 ? "FFW layer 1 launch" : "FFW layer 2 launch");
     }

@@ -44,6 +44,8 @@ constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at the boost 
 struct alignas(64) KernelParams {
     CUtensorMap tm_logits;  // [R, V], box 128 rows x (64 bytes of ids)
     CUtensorMap tm_E;       // [V, d], box kKBlock ids x 64 columns
+    CUtensorMap tm_out;     // pair kernel's TMA stores: z [R, d] bf16 (box 64 x 128) when splits == 1,
+                            // else the partial sums [splits, R, d] fp32 (box 32 x 128 x 1)
     const float* lse;
     uint16_t* z;
     float* partial;
@@ -56,10 +58,18 @@ struct alignas(64) KernelParams {
     float inv_tau[DG_MAX_CANVASES];
 };
 
-// GELU, tanh form (Hendrycks and Gimpel, "Gaussian Error Linear Units", 2016).
+// GELU, tanh form (Hendrycks and Gimpel, "Gaussian Error Linear Units", 2016), with the hardware
+// tanh approximation (tanh.approx.f32, relative error about 2^-11, below the bf16 rounding of the
+// result).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ float gelu_tanh(float x) {
     const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
-    return 0.5f * x * (1.0f + tanhf(k0 * fmaf(0.044715f * x, x * x, x)));
+    const float u = k0 * fmaf(0.044715f * x, x * x, x);
+    return 0.5f * x * (1.0f + tanh_approx(u));
 }
 
 // Eight fp32 accumulator values -> eight bf16 (16 bytes), with the epilogue activation.
@@ -290,6 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1) selfcond_kernel(const __grid_cons
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             int issued = 0;
+            // a plain operand may be the preceding grid's output (the FFW's hidden layer): wait for it
+            // (a no-op unless this is a programmatic dependent launch)
+            if (p.plain) grid_dependency_wait();
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
@@ -433,7 +446,13 @@ struct PairCfg {
     static constexpr int kEStagesFit = static_cast<int>((kBudget - kLStages * kLStageBytes) / kEBytes);
     static constexpr int kEStages = kEStagesFit > 16 ? 16 : kEStagesFit;
     static constexpr uint32_t kBarrierBytes = 1024;
-    static constexpr uint32_t kSmemBytes = kEStages * kEBytes + kLStages * kLStageBytes + kBarrierBytes + 1024;
+    static constexpr uint32_t kRingBytes = kEStages * kEBytes + kLStages * kLStageBytes;
+    static constexpr uint32_t kSmemBytes = kRingBytes + kBarrierBytes + 1024;
+    // epilogue: each of the two epilogue groups stages up to kSlabsPerGroup 16 KB slabs in the
+    // drained rings
+    static constexpr int kSlabsFit = static_cast<int>(kRingBytes / 2 / 16384u);
+    static constexpr int kSlabsPerGroup = kSlabsFit > 8 ? 8 : kSlabsFit;
+    static_assert(kSlabsPerGroup >= 1, "the rings must hold one epilogue slab per group");
     static_assert(kNT >= 128 && kNT % 128 == 0, "pair tiles hold whole 64-column boxes per CTA");
     static_assert(kEStages >= 4 && kLStages >= 2, "pipelines need depth");
     static_assert(kEBytes % 1024 == 0 && kLBytes % 1024 == 0 && kPBytes % 1024 == 0, "1 KB-aligned stage parts");
@@ -488,6 +507,85 @@ __device__ __forceinline__ void umma_commit_pair_both(uint32_t own_bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
                  ::"r"(own_bar), "h"(mask)
                  : "memory");
+}
+
+// Bulk tensor stores (shared memory -> global; completion tracked by bulk groups).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int32_t c0, int32_t c1, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tm), "r"(c0),
+                 "r"(c1), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, int32_t c0, int32_t c1, int32_t c2, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(tm), "r"(c0),
+                 "r"(c1), "r"(c2), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Barrier among the four warps of one epilogue group (named barrier 3 + group, 128 threads).
+__device__ __forceinline__ void epilogue_group_bar(int group) {
+    asm volatile("bar.sync %0, 128;" ::"r"(3 + group) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Epilogue of a CTA's 128-row accumulator by one group of four warps (all 128 rows, the group's half
+// of the kNT columns): TMEM -> registers -> activation and rounding -> shared memory -> TMA store.
+// A slab is 128 rows x 128 bytes (64 bf16 or 32 fp32 columns) in the 128-byte swizzle (16-byte
+// chunk c of row r at chunk position c ^ (r & 7)), so each warp's 16-byte stores spread over all
+// banks.  The group stages up to kSlabs slabs at a time in its part of the drained stage rings
+// (`area`), and its first thread (`issuer`) issues their stores.  Rows past R are clipped by the
+// tensor map; a CTA whose rows all lie past R stores nothing.
+template <int kNT, int kSlabs>
+__device__ void store_tile(const KernelParams& p, uint32_t tmem_lane_base, uint8_t* area, int group, int row,
+                           bool issuer, int32_t row0, int32_t col0, int split) {
+    constexpr int kHalf = kNT / 2;
+    const bool bf16_out = p.splits == 1;
+    const int cols_per_slab = bf16_out ? 64 : 32;
+    const int n_slabs = kHalf / cols_per_slab;
+    const uint32_t area_u32 = smem_u32(area);
+    const uint32_t row_base = area_u32 + static_cast<uint32_t>(row) * 128u;
+    const uint32_t sw = static_cast<uint32_t>(row & 7);
+    for (int b0 = 0; b0 < n_slabs; b0 += kSlabs) {
+        const int nb = min(kSlabs, n_slabs - b0);
+        if (b0 > 0) {  // the previous batch must have been read out before its slabs are overwritten
+            if (issuer) bulk_wait_read_all();
+            epilogue_group_bar(group);
+        }
+        for (int c = b0 * cols_per_slab; c < (b0 + nb) * cols_per_slab; c += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem_lane_base + static_cast<uint32_t>(group * kHalf + c), v);
+            const uint32_t slab_row = row_base + static_cast<uint32_t>(c / cols_per_slab - b0) * 16384u;
+            if (bf16_out) {
+                const uint32_t k0 = static_cast<uint32_t>((c % 64) / 8);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    st_shared_v4(slab_row + (((k0 + static_cast<uint32_t>(k)) ^ sw) << 4), pack8_act(v + 8 * k, p.act));
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    st_shared_v4(slab_row + ((static_cast<uint32_t>(k) ^ sw) << 4),
+                                 make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+            }
+        }
+        fence_proxy_async_smem();  // this thread's stores, visible to the bulk copies
+        epilogue_group_bar(group);
+        if (issuer && row0 < p.R) {
+            for (int j = 0; j < nb; ++j) {
+                const int32_t col = col0 + group * kHalf + (b0 + j) * cols_per_slab;
+                const uint32_t src = area_u32 + static_cast<uint32_t>(j) * 16384u;
+                if (bf16_out)
+                    tma_store_2d(&p.tm_out, col, row0, src);
+                else
+                    tma_store_3d(&p.tm_out, col, row0, split, src);
+            }
+            bulk_commit();
+        }
+    }
+    if (issuer) bulk_wait_all();  // complete before the CTA may exit
 }
 
 template <bool kBf16, int kNT>
@@ -588,6 +686,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             // Plain operands (bf16, used as loaded): both CTAs' tiles complete on the leader's barrier,
             // which the MMA thread waits on directly.
             const uint32_t leader_lfull0 = map_to_rank(smem_u32(&lfull[0]), 0);
+            // a plain operand may be the preceding grid's output (the FFW's hidden layer): wait for it
+            // (a no-op unless this is a programmatic dependent launch); the E copies need no wait
+            if (p.plain) grid_dependency_wait();
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kLS;
                 const uint32_t ph = (i / kLS) & 1;
@@ -671,30 +772,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (softmax_group_sync_or(group, !ok)) break;
             if (static_cast<int>(threadIdx.x) == leader_thread) mbar_arrive(&pready[s]);
         }
-        const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, wc));
+        // one exit decision per group: its warps meet at named barriers in the epilogue
+        const bool acc_fail = softmax_group_sync_or(group, !mbar_wait(accum, 0, wc));
         grid_launch_dependents();  // the split sum may launch; it waits for this grid's partials
-        if (acc_ok) {
+        if (!acc_fail) {
             tcgen05_after_sync();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            for (int c = group * (kNT / 2); c < (group + 1) * (kNT / 2); c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(lane_base + c, v);
-                if (valid) {
-                    const int32_t col = nt * kNT + c;
-                    if (p.splits == 1) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.z + static_cast<size_t>(r) * p.d + col);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = pack8_act(v + 8 * q, p.act);
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(
-                            p.partial + (static_cast<size_t>(split) * p.R + r) * p.d + col);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-                    }
-                }
-            }
+            const int32_t row0 = mp * 2 * kTileM + static_cast<int>(rank) * kTileM;
+            store_tile<kNT, G::kSlabsPerGroup>(p, lane_base, smem + group * G::kSlabsPerGroup * 16384, group, row,
+                                               static_cast<int>(threadIdx.x) == leader_thread, row0, nt * kNT, split);
         }
     }
 
@@ -729,6 +815,7 @@ __global__ void bounded_wait_test_kernel(long long limit) {
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ partial, uint2* __restrict__ z,
                                                             int64_t n4, int splits, int act) {
     grid_dependency_wait();  // launched dependent on the contraction: its partials must be complete
+    grid_launch_dependents();  // a dependent (the FFW's second layer) may be placed; it waits for this grid
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         // splits summed in order 0, 1, 2, ... (deterministic); loads issued eight at a time
@@ -802,6 +889,19 @@ cudaError_t encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base,
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_3d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, const uint64_t (&dims)[3],
+                      const uint64_t (&strides_bytes)[2], const uint32_t (&box)[3], CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+    const cuuint32_t b[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(tm, dt, 3, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Column tile: 512 when d allows; fp32 logits (small test workloads) stage twice the bytes per
 // tile and use at most 256 columns so that the pipeline keeps its depth.
 int pick_ntile(int d, bool logits_bf16) {
@@ -822,9 +922,9 @@ struct Plan {
     int ctas;
 };
 
-// Plain-operand GEMMs (the feed-forward block) are short in K: narrow column tiles give enough
-// tiles to fill the GPU without splitting K (and so without a split sum).
-int pick_ntile_plain(int d) { return d % 128 == 0 ? 128 : 64; }
+// Plain-operand GEMMs (the feed-forward block) are short in K: 256-column tiles (half the A-operand
+// re-reads of 128-column tiles) with a split of K that fills the GPU.
+int pick_ntile_plain(int d) { return d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64; }
 
 Plan plan(int R, int V, int d, bool logits_bf16, bool plain) {
     Plan pl;
@@ -925,6 +1025,17 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     e = encode_2d(&kp.tm_E, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.E, sp.d, sp.V, static_cast<uint64_t>(sp.d) * 2, 64,
                   kKBlock, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
+    if (pl.pair) {  // the pair kernel stores its tiles with TMA: z, or the split's partial sums
+        if (splits == 1)
+            e = encode_2d(&kp.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sp.z, sp.d, sp.R, static_cast<uint64_t>(sp.d) * 2,
+                          64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
+        else
+            e = encode_3d(&kp.tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.partial,
+                          {static_cast<uint64_t>(sp.d), static_cast<uint64_t>(sp.R), static_cast<uint64_t>(splits)},
+                          {static_cast<uint64_t>(sp.d) * 4, static_cast<uint64_t>(sp.R) * sp.d * 4},
+                          {32u, static_cast<uint32_t>(kTileM), 1u}, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+    }
     kp.lse = sp.lse;
     kp.z = sp.z;
     kp.partial = sp.partial;

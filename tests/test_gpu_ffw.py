@@ -51,7 +51,7 @@ def test_ffw_full_sampled_rows():
     _check(z, w1, w2, rows)
 
 
-@pytest.mark.parametrize("R,d,dff", [(200, 512, 2048), (1, 128, 512), (130, 256, 768)])
+@pytest.mark.parametrize("R,d,dff", [(200, 512, 2048), (1, 128, 512), (130, 256, 768), (300, 256, 512), (256, 384, 1152)])
 def test_ffw_edge_shapes(R, d, dff):
     g = torch.Generator(device=DEV).manual_seed(R + d)
     z = torch.randn(R, d, generator=g, device=DEV).to(torch.bfloat16)
