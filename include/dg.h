@@ -306,9 +306,11 @@ int dg_selfcond_drop(void* z, int32_t n_seq, int32_t C, int32_t d, uint64_t seed
 /* [d_ff, d]; hidden: device bf16 [rows, d_ff] (caller-owned scratch, also  */
 /* an output); z_out: device bf16 [rows, d]; all row-major, 16-byte aligned */
 /* and not aliased.  d, d_ff multiples of 64 in [64, 16384].  Workspace     */
-/* (256-byte aligned, zeroed before first use: it holds the split-K        */
-/* counters): dg_ffw_workspace_size bytes (may be 0).  Two contraction     */
-/* launches on `stream`.                                                    */
+/* (256-byte aligned, zeroed before first use like every workspace; it      */
+/* holds the layers' fp32 split-K partial sums): dg_ffw_workspace_size      */
+/* bytes (may be 0).  Up to four launches on `stream`: each layer's         */
+/* contraction and its split sum, the second layer a programmatic           */
+/* dependent of the first layer's last launch.                              */
 /* ------------------------------------------------------------------------ */
 size_t dg_ffw_workspace_size(int32_t rows, int32_t d, int32_t d_ff);
 
