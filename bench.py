@@ -81,12 +81,39 @@ def whole_job_rate(local_ms: float, units_per_rank: int, world: int, device="cpu
 
 
 # ------------------------------------------------------------------------------ clocks
+# NVML poller run as a child process (no GIL shared with the timing thread): prints
+# "time sm_mhz max_sm_mhz reason_bits" lines about every 0.2 ms until it is terminated.
+_NVML_POLLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+out = sys.stdout
+while True:
+    out.write("%.6f %d %d %d\n" % (time.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                    int(reasons(h))))
+    out.flush()
+    time.sleep(0.0002)
+"""
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled while the timed region runs.
+
+    An NVML poller in a child process samples about every 0.2 ms; the samples kept are those whose
+    time lies between mark_start() and mark_end(), which bracket the timed region, so even a region
+    of a few milliseconds is sampled from inside.  Without NVML: nvidia-smi every 200 ms around the
+    region."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
         self.gpu = str(gpu_index)
@@ -98,17 +125,48 @@ class ClockSampler:
             pass
         self.proc = None
         self.lines = []
+        self.nvml = False
+        self.samples = []  # (time, sm MHz, max sm MHz, reason bits) from NVML
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml  # noqa: F401  (the poller needs it)
+        except ImportError:
+            return False
+        try:
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLLER, self.gpu], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return False
+        first = self.proc.stdout.readline()  # wait until it samples
+        if not first:
+            self.proc.wait(timeout=5)
+            self.proc = None
+            return False
+        self.lines.append(first.strip())
+        return True
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        self.nvml = self._start_nvml()
+        if not self.nvml:
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+        if self.proc is not None:
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+        if not self.nvml:
+            time.sleep(0.3)
         return self
 
     def _read(self):
@@ -116,33 +174,54 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
-        time.sleep(0.25)
+        time.sleep(0.01 if self.nvml else 0.25)
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.thread.join(timeout=5)
+        if self.nvml:
+            for line in self.lines:
+                f = line.split()
+                if len(f) == 4:
+                    try:
+                        self.samples.append((float(f[0]), float(f[1]), float(f[2]), int(f[3])))
+                    except ValueError:
+                        pass
 
     def summary(self):
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
+        if self.nvml:
+            for t, clk, m, bits in self.samples:
+                if self.t0 is not None and t < self.t0:
+                    continue
+                if self.t1 is not None and t > self.t1:
+                    continue
+                sm.append(clk)
+                mx.append(m)
+                reasons.update(name for name, bit in self.REASON_BITS.items() if bits & bit)
+            src = "nvml (child process, every ~0.2 ms), samples inside the timed region"
+        else:
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in self.lines:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, f[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+            src = "nvidia-smi every 200 ms around the timed region"
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": src}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": src}
 
 
 # ------------------------------------------------------------------------------ roofline helpers
@@ -201,6 +280,12 @@ def timed_replay(g, stream) -> float:
         b.record(stream)
     stream.synchronize()
     return a.elapsed_time(b)
+
+
+def settle(stream, seconds: float = 0.5) -> None:
+    """Idle the GPU briefly between independent measurement blocks."""
+    stream.synchronize()
+    time.sleep(seconds)
 
 
 def run_ours(args, rank, world, local):
@@ -275,11 +360,13 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     with ClockSampler(local) as clocks:
+        clocks.mark_start()
         with torch.cuda.stream(stream):
             ev[0].record(stream)
             g_steps.replay()
             ev[1].record(stream)
         stream.synchronize()
+        clocks.mark_end()
     torch.cuda.synchronize(dev)
     barrier()
     total_ms = ev[0].elapsed_time(ev[1])
@@ -287,6 +374,7 @@ def run_ours(args, rank, world, local):
     total_ms, steps_per_s = whole_job_rate(total_ms, K, world, dev)
 
     # ---- the two kernels of the step, each in a graph of K back-to-back launches (same inputs)
+    settle(stream)
     for g in (g_k1, g_k2):
         timed_replay(g, stream)  # warm
     k1_us = timed_replay(g_k1, stream) * 1e3 / K
@@ -317,10 +405,16 @@ def run_ours(args, rank, world, local):
         roof["tensor_frac_sustained"] = round(tflops / peaks["bf16_tflops_sustained"], 4)
     k1_gbs = bytes_k1 / (k1_us * 1e-6) / 1e9
 
-    # ---- training-side kernels, entropy-bounded step, FFW, other workloads
+    # ---- training-side kernels, entropy-bounded step, FFW, other workloads.  Each block starts after a
+    # short idle gap, so that the power controller's state after the previous block's load (the SM
+    # clock it settled at under the 1 kW cap) does not carry into the next block's numbers.
+    settle(stream)
     train = bench_train(dg, W, dev, stream, hbm)
+    settle(stream)
     eb = bench_eb(dg, W, dev, stream, bufs, hbm)
+    settle(stream)
     ffw = bench_ffw(dg, W, dev, stream, peaks)
+    settle(stream)
     configs = bench_configs(dg, W, dev, stream, peaks)
 
     # ---- end to end through the public API with host buffers
@@ -788,8 +882,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=120)
-    ap.add_argument("--warmup", type=int, default=12)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

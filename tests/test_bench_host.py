@@ -49,6 +49,16 @@ def test_clock_summary_parses_samples():
     assert s["reasons"] == ["sw_power_cap"]
     empty = bench.ClockSampler(0)
     assert empty.summary()["samples"] == 0
+    # NVML samples: (time, SM MHz, max SM MHz, clock-event reason bits); only those inside the region
+    nv = bench.ClockSampler(0)
+    nv.nvml = True
+    nv.samples = [(0.5, 900, 1965, 0x1), (1.0, 1965, 1965, 0x1), (1.1, 1500, 1965, 0x4),
+                  (1.2, 1400, 1965, 0x4 | 0x40), (1.3, 1600, 1965, 0x0), (2.5, 1965, 1965, 0x8)]
+    nv.t0, nv.t1 = 1.0, 2.0
+    s = nv.summary()
+    assert s["samples"] == 4 and s["sm_mhz"] == 1550 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]  # 0x1 (idle) is not a slowdown
+    assert s["source"].startswith("nvml")
 
 
 def test_oracle_sample_single_and_threaded_on_tiny():
