@@ -51,10 +51,30 @@ def test_ffw_full_sampled_rows():
     _check(z, w1, w2, rows)
 
 
-@pytest.mark.parametrize("R,d,dff", [(200, 512, 2048), (1, 128, 512), (130, 256, 768), (300, 256, 512), (256, 384, 1152)])
+@pytest.mark.parametrize("R,d,dff", [(200, 512, 2048), (1, 128, 512), (130, 256, 768), (300, 256, 512), (256, 384, 1152),
+                                      (200, 512, 8192)])  # two K-splits folded, ragged rows
 def test_ffw_edge_shapes(R, d, dff):
     g = torch.Generator(device=DEV).manual_seed(R + d)
     z = torch.randn(R, d, generator=g, device=DEV).to(torch.bfloat16)
     w1 = (torch.randn(d, dff, generator=g, device=DEV) * d ** -0.5).to(torch.bfloat16)
     w2 = (torch.randn(dff, d, generator=g, device=DEV) * dff ** -0.5).to(torch.bfloat16)
     _check(z, w1, w2)
+
+
+def test_ffw_repeated_calls_one_workspace():
+    # Successive calls on one workspace: the first layer's two K-splits hand their partial tiles over
+    # through counters in the workspace, which the second layer's partial sums must not disturb.
+    cfg = W.FULL
+    z, w1, w2 = W.make_ffw(cfg, DEV)
+    R, d = z.shape
+    dff = w1.shape[1]
+    ws = torch.zeros(max(256, int(dg.lib().dg_ffw_workspace_size(R, d, dff))), dtype=torch.uint8, device=DEV)
+    rows = np.sort(np.random.default_rng(1).choice(R, 6, replace=False))
+    a, b = w1.float().cpu().numpy(), w2.float().cpu().numpy()
+    for k in range(3):
+        zk = (z.float() * (1.0 + 0.5 * k) - 0.25 * k).to(torch.bfloat16)
+        out, _ = dg.dg_ffw(zk, w1, w2, ws=ws)
+        torch.cuda.synchronize()
+        ref = O.ffw(zk.float().cpu().numpy()[rows], a, b)
+        assert rel_fro(out.float().cpu().numpy()[rows], ref) <= TOL, k
+    assert dg.dg_device_error() == 0

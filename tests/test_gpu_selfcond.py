@@ -125,6 +125,7 @@ def test_batched_sampled_rows_and_mass():
     (64, 64, 777, 784, 256, torch.bfloat16, torch.float32),
     (129, 43, 3000, 3000, 1536, torch.bfloat16, torch.bfloat16),
     (300, 100, 3001, 3008, 256, torch.bfloat16, torch.bfloat16),  # a pair CTA with every row past R
+    (256, 128, 1000, 1000, 16384, torch.bfloat16, torch.bfloat16),  # two K-splits folded (no split sum)
     (1, 1, 33, 40, 512, torch.float32, torch.float32),
     (6, 3, (1 << 20) + 3, (1 << 20) + 8, 64, torch.bfloat16, torch.bfloat16),  # rows past 512 chunks
 ])
