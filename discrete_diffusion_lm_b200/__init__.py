@@ -40,7 +40,9 @@ from typing import Optional, Sequence
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdg.so")
+# DG_LIB=checks selects the checks library (device-side index and token-id checks, built with
+# `python -m discrete_diffusion_lm_b200.build --checks`); anything else, or unset, the normal one.
+LIB_PATH = os.path.join(_PKG, "libdg_checks.so" if os.environ.get("DG_LIB") == "checks" else "libdg.so")
 
 DG_OK = 0
 DG_F32, DG_BF16 = 0, 1
@@ -68,7 +70,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m discrete_diffusion_lm_b200.build`")
+            flag = " --checks" if LIB_PATH.endswith("_checks.so") else ""
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m discrete_diffusion_lm_b200.build{flag}`")
         L = ctypes.CDLL(LIB_PATH)
         L.dg_last_error.restype = ctypes.c_char_p
         L.dg_version.restype = ctypes.c_char_p

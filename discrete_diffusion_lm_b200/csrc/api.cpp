@@ -193,11 +193,15 @@ int dg_device_error(int* code) {
     if ((rc = check_device()) != DG_OK) return rc;
     const cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    int c1 = 0, c2 = 0;
-    cudaError_t r = read_and_clear_device_error(&c1);
-    if (r == cudaSuccess) r = read_and_clear_pass_error(&c2);
+    int c[4] = {0, 0, 0, 0};
+    cudaError_t r = read_and_clear_device_error(&c[0]);
+    if (r == cudaSuccess) r = read_and_clear_pass_error(&c[1]);
+    if (r == cudaSuccess) r = read_and_clear_ops_error(&c[2]);
+    if (r == cudaSuccess) r = read_and_clear_noise_error(&c[3]);
     if (r != cudaSuccess) return cuda_fail(r, "reading the device error words");
-    *code = c1 ? c1 : c2;
+    *code = 0;
+    for (int k = 0; k < 4; ++k)  // the largest code: a failed check (2) before an expired wait (1)
+        if (c[k] > *code) *code = c[k];
     return DG_OK;
 }
 

@@ -21,6 +21,11 @@
 
 namespace dg {
 
+// Device error word of the per-canvas decisions and the other kernels of canvas_ops.cu (the one
+// translation unit that includes this header): code 2 from a failed device-side check (checks
+// library only).  Read and cleared by dg_device_error.
+__device__ int g_ops_error = 0;
+
 // Shared-memory scratch of one canvas's decisions (C up to DG_MAX_CANVAS_ROWS): the sorted 32-key
 // chunks, the rank-ordered q, each position's rank, and the block reductions' slots.
 static_assert(DG_MAX_CANVAS_ROWS <= 1024, "positions must fit the key's low 10 bits");
@@ -148,8 +153,10 @@ __device__ void decide_canvas(const DecideParams& p, int b, DecideShared& sh) {
             int r = 0;  // the own chunk contributes the key's lane: keys are unique
 #pragma unroll 4
             for (int c = 0; c < n_chunks; ++c) r += count_below32(sh.chunks + c * 32, key[u]);
-            sh.sorted[r] = static_cast<long long>(key[u] >> 10);
-            sh.rank[key[u] & 1023u] = r;
+            if (DG_CHECKED(g_ops_error, r < C && static_cast<int>(key[u] & 1023u) < C)) {
+                sh.sorted[r] = static_cast<long long>(key[u] >> 10);
+                sh.rank[key[u] & 1023u] = r;
+            }
         }
     }
     __syncthreads();
@@ -186,6 +193,7 @@ __device__ void decide_canvas(const DecideParams& p, int b, DecideShared& sh) {
             const int64_t r = r0 + i;
             const bool acc = sh.rank[i] < n_acc;
             int32_t x = x0[u];
+            if (acc) DG_CHECK(g_ops_error, x >= 0 && x < p.V);  // an x0_hat the caller gave
             if (!acc) {
                 const uint4 w =
                     philox4x32_10(make_uint4(0u, static_cast<uint32_t>(r), p.step, kDomRenoise), p.key0, p.key1);

@@ -44,7 +44,10 @@ __global__ void __launch_bounds__(256) ce_backward_kernel(const __grid_constant_
         const int32_t b = r / p.C, i = r - b * p.C;
         const int32_t k = p.canvas_idx[b];
         int32_t y = -1;
+        if (threadIdx.x == 0 && blockIdx.x == 0) DG_CHECK(g_ops_error, k >= 0 && k < p.K);  // caller's index
         if (k >= 0 && k < p.K) y = p.x0[static_cast<int64_t>(b) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i];
+        if (threadIdx.x == 0 && blockIdx.x == 0 && k >= 0 && k < p.K)
+            DG_CHECK(g_ops_error, y >= 0 && y < p.V);  // a token id the caller gave
         uint4* row = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.logits) + static_cast<int64_t>(r) * p.ld);
         const int32_t v_base = blockIdx.x * (kCeVec * 256) + threadIdx.x;
         if (y < 0 || y >= p.V) {
@@ -99,6 +102,18 @@ __global__ void __launch_bounds__(256) selfcond_drop_kernel(uint16_t* z, int64_t
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_ops_error(int* out) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_ops_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_ops_error, &zero, sizeof(int));
+    }
+    *out = v;
+    return e;
+}
 
 cudaError_t launch_canvas_decide(const DecideParams& p, int32_t B, cudaStream_t s) {
     if (B < 1 || p.C < 1 || p.C > DG_MAX_CANVAS_ROWS) return cudaErrorInvalidValue;

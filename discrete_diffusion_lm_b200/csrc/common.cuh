@@ -13,6 +13,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegBig = -1.0e30f;  // -inf logits are clamped here before any arithmetic
 
+// Device-side checks, compiled in by the checks library (DG_CHECKS=1) and away otherwise.
+//   DG_CHECK(word, cond)    statement: when cond fails, code 2 goes to the device error word;
+//   DG_CHECKED(word, cond)  expression guarding an access: the same, and false skips the access.
+// In the normal build cond is not evaluated: DG_CHECK is a no-op and DG_CHECKED is true.
+#if defined(DG_CHECKS) && DG_CHECKS
+#define DG_CHECK(word, cond)          \
+    do {                              \
+        if (!(cond)) atomicMax(&(word), 2); \
+    } while (0)
+#define DG_CHECKED(word, cond) ((cond) ? true : (atomicMax(&(word), 2), false))
+#else
+#define DG_CHECK(word, cond) ((void)0)
+#define DG_CHECKED(word, cond) true
+#endif
+
 // ---------------------------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
 // SC'11): ten rounds; each multiplies counter words 0 and 2 by the two published multipliers,

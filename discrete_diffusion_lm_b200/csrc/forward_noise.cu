@@ -18,6 +18,10 @@ namespace dg {
 
 namespace {
 
+// Device error word of this file's kernel: code 2 from a failed device-side check (checks library
+// only).  Read and cleared by dg_device_error.
+__device__ int g_noise_error = 0;
+
 constexpr int kNoiseThreads = 256;
 
 __global__ void __launch_bounds__(kNoiseThreads) forward_noise_kernel(const __grid_constant__ NoiseParams p) {
@@ -30,6 +34,7 @@ __global__ void __launch_bounds__(kNoiseThreads) forward_noise_kernel(const __gr
     if (j >= p.seq_len) return;
     const int64_t at = static_cast<int64_t>(b) * p.seq_len + j;
     int32_t tok = p.x0[at];
+    DG_CHECK(g_noise_error, tok >= 0 && tok < p.V);  // a token id the caller gave
     if (j >= p.P) {
         const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(j), static_cast<uint32_t>(b), 0u, kDomNoise),
                                       p.key0, p.key1);
@@ -39,6 +44,18 @@ __global__ void __launch_bounds__(kNoiseThreads) forward_noise_kernel(const __gr
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_noise_error(int* out) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_noise_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_noise_error, &zero, sizeof(int));
+    }
+    *out = v;
+    return e;
+}
 
 cudaError_t launch_forward_noise(const NoiseParams& p, cudaStream_t s) {
     const long long bx = (p.seq_len + kNoiseThreads - 1) / kNoiseThreads;

@@ -100,6 +100,9 @@ cudaError_t launch_convert_f32_bf16(const float* in, uint16_t* out, int64_t n, c
 cudaError_t launch_bounded_wait_test(long long limit_cycles, cudaStream_t s);
 // Reads (synchronously) and clears the error word set by a kernel whose bounded wait expired.
 cudaError_t read_and_clear_device_error(int* out);
+// The same for the error words of canvas_ops.cu and forward_noise.cu (device-side checks).
+cudaError_t read_and_clear_ops_error(int* out);
+cudaError_t read_and_clear_noise_error(int* out);
 
 // Per-canvas sampler decisions: entropy-bounded acceptance with uniform re-noising, and the
 // adaptive-stopping flag.  One CTA per canvas.  Null outputs skip their part (x_next == nullptr:

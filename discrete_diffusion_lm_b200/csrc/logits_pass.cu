@@ -399,7 +399,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
                 for (int k = 0; k < 4 && j + k < nch; ++k) (void)get_record<kBf16>(rec, j + k, tag, ready);
             if (ready) break;
             if (clock64() - t0 > limit) {
-                atomicExch(&g_pass_error, 1);
+                atomicMax(&g_pass_error, 1);
                 break;
             }
             __nanosleep(64);
@@ -414,9 +414,11 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         b_seq = row / p.C;
         i_seq = row - b_seq * p.C;
         const int32_t k = p.canvas_idx[b_seq];
+        DG_CHECK(g_pass_error, k >= 0 && k < p.K);  // a canvas index the caller gave
         if (k >= 0 && k < p.K) {
             const int32_t target =
                 p.x0[static_cast<int64_t>(b_seq) * p.seq_len + p.P + static_cast<int64_t>(k) * p.C + i_seq];
+            DG_CHECK(g_pass_error, target >= 0 && target < p.V);  // a token id the caller gave
             if (target >= 0 && target < p.V) {
                 target_logit = load_logit(rowp, target, kBf16);
                 target_ok = true;
@@ -438,6 +440,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
     if (kKind == kPassSampler && tid == 0) asm volatile("" ::"l"(out_x0), "l"(out_am), "l"(out_mp), "l"(out_lse), "l"(out_h));
     if (kKind == kPassSampler && tid == 0 && p.x_next) {
         xt = p.x_t[row];
+        DG_CHECK(g_pass_error, xt >= 0 && xt < p.V);  // a token id the caller gave
         thr_sd = p.thr_stay_diff[canvas];
         thr_jd = p.thr_jump_diff[canvas];
         thr_ss = p.thr_stay_same[canvas];
@@ -505,6 +508,8 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
 
     const float m_raw = acc.mv;
     int32_t jm = acc.jm, bj = acc.bj;
+    DG_CHECK(g_pass_error, jm < nch);                                 // NaN logits only
+    DG_CHECK(g_pass_error, !sampling || !(acc.S > 0.f) || bj < nch);  // likewise
     if (jm >= nch) jm = 0;  // only reachable with NaN inputs; keeps every index in range
     if (!sampling || bj >= nch) bj = jm;  // greedy, or NaN scores only
     const float m_row = m_raw * inv_tau;
@@ -614,6 +619,7 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
         }
     }
     block_argmax2<kPassWarps>(amv, am, bs2, bv, sh.f, sh.i);
+    DG_CHECK(g_pass_error, am >= alo && am < ahi);  // NaN logits only
     if (am < alo || am >= ahi) am = alo;
     const int32_t x0 = sampling && bv >= glo && bv < ghi ? bv : am;
 
@@ -641,11 +647,11 @@ __device__ __noinline__ void merge_row(const PassParams& p, int32_t row, int32_t
                 xn = word_to_index(w.y, p.V);
                 br = 2;
             }
-            p.x_next[row] = xn;
+            if (DG_CHECKED(g_pass_error, xn >= 0 && xn < p.V)) p.x_next[row] = xn;
             if (p.branch) p.branch[row] = br;
         }
-        if (out_x0) out_x0[row] = x0;
-        if (out_am) out_am[row] = am;
+        if (out_x0 && DG_CHECKED(g_pass_error, (x0 >= alo && x0 < ahi) || (x0 >= glo && x0 < ghi))) out_x0[row] = x0;
+        if (out_am && DG_CHECKED(g_pass_error, am >= 0 && am < p.V)) out_am[row] = am;
         if (out_mp) out_mp[row] = 1.0f / S;
         if (out_lse) out_lse[row] = lse;
         if (out_h) out_h[row] = ln_s - T / S;

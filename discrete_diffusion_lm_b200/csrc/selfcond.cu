@@ -114,7 +114,7 @@ __device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, Wait
         if (aborted(ctl)) return false;
         if (clock64() - t0 > ctl->limit) {
             *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
-            atomicExch(&g_device_error, 1);
+            atomicMax(&g_device_error, 1);
             return false;
         }
     }
@@ -577,6 +577,7 @@ __device__ void store_tile(const KernelParams& p, uint32_t tmem_lane_base, uint8
             for (int j = 0; j < nb; ++j) {
                 const int32_t col = col0 + group * kHalf + (b0 + j) * cols_per_slab;
                 const uint32_t src = area_u32 + static_cast<uint32_t>(j) * 16384u;
+                if (!DG_CHECKED(g_device_error, col >= 0 && col + cols_per_slab <= p.d)) continue;
                 if (bf16_out)
                     tma_store_2d(&p.tm_out, col, row0, src);
                 else
@@ -665,6 +666,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
                     for (int j = 0; j < G::kBoxesPerHalf; ++j) {
                         const int col = nt * kNT + nh * G::kMmaN + static_cast<int>(rank) * (G::kMmaN / 2) + 64 * j;
+                        DG_CHECK(g_device_error, col + 64 <= p.d && k0 < p.V);
                         tma_load_2d_pair(dst + (nh * G::kBoxesPerHalf + j) * (64 * kKBlock * 2), &p.tm_E, col, k0,
                                          leader_efull0 + s * 8);
                     }

@@ -102,10 +102,14 @@ const char* dg_version(void);
 /* Number of kernels this library has launched in this process so far. */
 uint64_t dg_launch_count(void);
 /* Synchronizes the current device, then stores in *code (and clears) the
- * library's device error word: 0 if no kernel has reported a problem, 1 if a
- * kernel gave up on a bounded wait (its outputs are then incomplete).  Every
- * wait inside the library's kernels is bounded (about two seconds), so a
- * stalled pipeline ends with this code instead of hanging the device. */
+ * library's device error words (the largest code they hold): 0 if no kernel
+ * has reported a problem, 1 if a kernel gave up on a bounded wait (its
+ * outputs are then incomplete), 2 if a device-side check failed.  Every wait
+ * inside the library's kernels is bounded (about two seconds), so a stalled
+ * pipeline ends with code 1 instead of hanging the device.  Code 2 comes only
+ * from the checks build of the library (libdg_checks.so, DG_CHECKS=1), whose
+ * kernels verify the token ids and canvas indices they are given and their
+ * own index invariants, and skip an access that would fail a check. */
 int dg_device_error(int* code);
 
 /* ------------------------------------------------------------------------ */

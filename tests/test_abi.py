@@ -235,3 +235,14 @@ def test_binding_constants_match_the_header():
     for name in ("DG_GUMBEL_CHUNK", "DG_MAX_CANVASES", "DG_MAX_CANVAS_ROWS", "DG_MAX_VOCAB",
                  "DG_NOALLOC_SCRATCH_BYTES"):
         assert getattr(dg, name) == _int_expr(defines[name]), name
+
+
+def test_checks_library_builds_and_exports_the_same_symbols():
+    # the checks build (DG_CHECKS=1): same sources and entry points, device-side checks compiled in
+    path = build.build(checks=True)
+    assert path.endswith("libdg_checks.so") and os.path.exists(path)
+    C = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(C, n), n
+    C.dg_version.restype = ctypes.c_char_p
+    assert C.dg_version() == dg.lib().dg_version()
