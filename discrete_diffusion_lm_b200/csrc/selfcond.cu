@@ -814,6 +814,47 @@ __global__ void bounded_wait_test_kernel(long long limit) {
 }
 
 // z[i] = bf16(sum_s partial[s][i]) in a fixed order (deterministic).
+// Few splits (the FFW's first layer has two): each thread takes kPos positions a stride apart and
+// issues all their loads before the first add, so a thread's positions cost one memory round trip.
+template <int kPos, int kMaxS>
+__global__ void __launch_bounds__(256) splitk_reduce_few_kernel(const float4* __restrict__ partial,
+                                                                uint2* __restrict__ z, int64_t n4, int splits,
+                                                                int act) {
+    grid_dependency_wait();  // launched dependent on the contraction: its partials must be complete
+    grid_launch_dependents();  // a dependent (the FFW's second layer) may be placed; it waits for this grid
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n4; i0 += kPos * stride) {
+        float4 v[kPos][kMaxS];
+#pragma unroll
+        for (int q = 0; q < kPos; ++q)
+#pragma unroll
+            for (int s = 0; s < kMaxS; ++s)
+                if (s < splits && i0 + q * stride < n4)
+                    v[q][s] = __ldcs(partial + static_cast<int64_t>(s) * n4 + i0 + q * stride);
+#pragma unroll
+        for (int q = 0; q < kPos; ++q) {
+            const int64_t i = i0 + q * stride;
+            if (i >= n4) continue;
+            float4 acc = v[q][0];  // splits summed in order 0, 1, ... (deterministic)
+#pragma unroll
+            for (int s = 1; s < kMaxS; ++s)
+                if (s < splits) {
+                    acc.x += v[q][s].x;
+                    acc.y += v[q][s].y;
+                    acc.z += v[q][s].z;
+                    acc.w += v[q][s].w;
+                }
+            if (act) {
+                acc.x = gelu_tanh(acc.x);
+                acc.y = gelu_tanh(acc.y);
+                acc.z = gelu_tanh(acc.z);
+                acc.w = gelu_tanh(acc.w);
+            }
+            z[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ partial, uint2* __restrict__ z,
                                                             int64_t n4, int splits, int act) {
     grid_dependency_wait();  // launched dependent on the contraction: its partials must be complete
@@ -1091,8 +1132,15 @@ cudaError_t launch_selfcond(const SelfcondParams& sp, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, reinterpret_cast<const float4*>(sp.partial),
-                           reinterpret_cast<uint2*>(sp.z), n4, splits, static_cast<int>(sp.act));
+    if (splits == 2)
+        e = cudaLaunchKernelEx(&cfg, splitk_reduce_few_kernel<4, 2>, reinterpret_cast<const float4*>(sp.partial),
+                               reinterpret_cast<uint2*>(sp.z), n4, splits, static_cast<int>(sp.act));
+    else if (splits <= 4)
+        e = cudaLaunchKernelEx(&cfg, splitk_reduce_few_kernel<2, 4>, reinterpret_cast<const float4*>(sp.partial),
+                               reinterpret_cast<uint2*>(sp.z), n4, splits, static_cast<int>(sp.act));
+    else
+        e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, reinterpret_cast<const float4*>(sp.partial),
+                               reinterpret_cast<uint2*>(sp.z), n4, splits, static_cast<int>(sp.act));
     if (e != cudaSuccess) return e;
     note_launches(1);
     return cudaGetLastError();
