@@ -5,8 +5,12 @@ step) with V from 1 to 9000 (chunk multiples and their neighbours among them), r
 logits of random scale with a few large peaks and a few masked (-inf) ids per row; the comparison
 is tests/parity.py's: exact argmax, statistics within 1e-3, x0_hat and x_next exact off near-ties.
 Contraction: 12 draws of (R, C, V, d, logits dtype, embedding dtype) with per-canvas inv_tau, z on
-sampled rows within the per-row relative Frobenius bound.  The draws come from a fixed numpy seed,
-so every run checks the same cases.
+sampled rows within the per-row relative Frobenius bound.  Decisions: 16 draws of (B, C up to 1024,
+entropy kind -- continuous, heavily tied, below the fixed-point resolution, with NaN / negative /
+large values --, tolerance, threshold, with or without a previous argmax canvas), bit-exact against
+the oracle.  Training side: 12 draws of (n_seq, P, K, C, V, dtype, schedule), forward corruption
+bit-exact and the canvas cross-entropy within its tolerances.  The draws come from fixed numpy
+seeds, so every run checks the same cases.
 """
 import numpy as np
 import pytest
@@ -105,4 +109,88 @@ def test_selfcond_random_shapes(case):
     zr = O.selfcond_rows(host_f32(L)[:, :ld], host_f32(E), rows, it_rows)
     err = rel_fro_rows(z.float().cpu().numpy()[rows], zr)
     assert err.max() <= Z_REL_FRO, (case, err.max())
+    assert dg.dg_device_error() == 0
+
+
+def _decision_cases():
+    rng = np.random.default_rng(4242)
+    cases = []
+    for i in range(16):
+        cases.append(dict(i=i, B=int(rng.integers(1, 9)), C=int(rng.integers(1, 1025)),
+                          kind=str(rng.choice(["uniform", "tied", "tiny", "special"])),
+                          eps_frac=float(rng.choice([0.0, 0.1, 0.5, 1.0, 2.0])), theta=float(rng.uniform(0, 3)),
+                          prev=bool(rng.random() < 0.7), rng_seed=int(rng.integers(0, 2 ** 31))))
+    return cases
+
+
+def _entropies(kind, n, rng):
+    if kind == "uniform":
+        return rng.uniform(0.0, 6.0, n).astype(np.float32)
+    if kind == "tied":
+        return rng.choice(np.float32([0.0, 0.25, 1.0, 2.5]), n).astype(np.float32)
+    if kind == "tiny":
+        return (rng.uniform(0, 4, n) * 2.0 ** -33).astype(np.float32)
+    h = rng.uniform(0.0, 3.0, n).astype(np.float32)  # special values
+    for v in (np.nan, -1e-6, 90.0):
+        h[rng.integers(0, n, max(1, n // 16))] = v
+    return h
+
+
+@pytest.mark.parametrize("case", _decision_cases(), ids=lambda c: f"d{c['i']}")
+def test_decisions_random(case):
+    rng = np.random.default_rng(case["rng_seed"])
+    B, C, V = case["B"], case["C"], 262144
+    H = _entropies(case["kind"], B * C, rng)
+    x0 = rng.integers(0, V, B * C).astype(np.int32)
+    eps = case["eps_frac"] * float(np.nansum(np.clip(H[:C], 0, 64)))
+    seed, step = int(rng.integers(0, 2 ** 40)), int(rng.integers(0, 1000))
+    Hd = torch.from_numpy(H).to(DEV)
+    acc = dg.dg_entropy_accept(Hd, torch.from_numpy(x0).to(DEV), C, V, eps, seed=seed, step=step)
+    am = rng.integers(0, V, B * C).astype(np.int32)
+    prev = am.copy()
+    prev[rng.integers(0, B * C, max(1, B // 2))] += 1  # some canvases changed their prediction
+    p = prev if case["prev"] else None
+    stop, mean = dg.dg_adaptive_stop(Hd, torch.from_numpy(am).to(DEV), None if p is None else torch.from_numpy(p).to(DEV),
+                                     C, case["theta"])
+    torch.cuda.synchronize()
+    x_ref, a_ref, n_ref = O.entropy_accept(H, x0, B, C, V, eps, seed, step)
+    np.testing.assert_array_equal(acc["accepted"].cpu().numpy(), a_ref)
+    np.testing.assert_array_equal(acc["n_accepted"].cpu().numpy(), n_ref)
+    np.testing.assert_array_equal(acc["x_next"].cpu().numpy(), x_ref)
+    s_ref, m_ref = O.adaptive_stop(H, am, p, B, C, case["theta"])
+    np.testing.assert_array_equal(stop.cpu().numpy(), s_ref)
+    np.testing.assert_array_equal(mean.cpu().numpy(), m_ref.astype(np.float32))
+
+
+def _train_cases():
+    rng = np.random.default_rng(99)
+    return [dict(i=i, n_seq=int(rng.integers(1, 7)), P=int(rng.integers(0, 65)), K=int(rng.integers(1, 5)),
+                 C=int(rng.integers(1, 65)), V=int(rng.integers(1, 5001)),
+                 dtype=torch.bfloat16 if rng.random() < 0.6 else torch.float32,
+                 schedule=str(rng.choice(["linear", "cosine"])), rng_seed=int(rng.integers(0, 2 ** 31)))
+            for i in range(12)]
+
+
+@pytest.mark.parametrize("case", _train_cases(), ids=lambda c: f"t{c['i']}")
+def test_forward_noise_and_canvas_ce_random(case):
+    rng = np.random.default_rng(case["rng_seed"])
+    n_seq, P, K, C, V = case["n_seq"], case["P"], case["K"], case["C"], case["V"]
+    x0 = torch.from_numpy(rng.integers(0, V, (n_seq, P + K * C)).astype(np.int32)).to(DEV)
+    t = list(rng.uniform(0.0, 1.0, n_seq))
+    seed = int(rng.integers(0, 2 ** 40))
+    xt, kk = dg.dg_forward_noise(x0, P, K, C, V, t, schedule=case["schedule"], seed=seed)
+    torch.cuda.synchronize()
+    rx, rk = O.forward_noise(x0.cpu().numpy(), n_seq, P, K, C, V, case["schedule"], t, seed)
+    np.testing.assert_array_equal(xt.cpu().numpy(), rx)
+    np.testing.assert_array_equal(kk.cpu().numpy(), rk)
+    elt = 2 if case["dtype"] == torch.bfloat16 else 4
+    L = _logits(n_seq * C, V, _padded(V, elt, rng), case["dtype"], rng)
+    loss, seq, lse = dg.dg_canvas_ce(L, x0, kk, P, K, C, V=V)
+    torch.cuda.synchronize()
+    rl, rs, rlse = O.canvas_ce(host_f32(L), x0.cpu().numpy(), kk.cpu().numpy(), n_seq, P, K, C, V)
+    gl = loss.cpu().numpy().astype(np.float64)
+    with np.errstate(invalid="ignore"):  # a masked (-inf) target gives +inf loss on both sides
+        assert np.all((gl == rl) | (np.abs(gl - rl) <= 1e-3 + 1e-5 * np.abs(rl))), case
+    assert np.all(np.abs(lse.cpu().numpy() - rlse) <= 1e-3), case
+    np.testing.assert_allclose(seq.cpu().numpy(), rs, rtol=1e-5, atol=1e-2)
     assert dg.dg_device_error() == 0

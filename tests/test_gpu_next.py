@@ -100,15 +100,15 @@ def test_sampler_step_eb_equals_its_parts():
 
 
 def test_sampler_step_eb_batched_equals_its_parts():
-    # 16 canvases with per-canvas temperatures: the decisions run in the merge of each canvas's
-    # last row and must equal the standalone decisions on the same outputs
+    # 16 canvases with per-canvas temperatures: the step's decisions (its decision kernel after the
+    # pass) must equal the standalone decisions on the same outputs
     cfg = W.BATCHED
     rows = 16 * 256
     logits = W.make_logits(cfg, DEV, rows=rows)
     ts = [1.0 - b / 16 for b in range(16)]
     inv_tau = dg.dg_tau_linear(ts)
     prev = torch.from_numpy(np.random.default_rng(1).integers(0, cfg.V, rows).astype(np.int32)).to(DEV)
-    for rep in range(2):  # the canvas tickets must be back at zero for the second call
+    for rep in range(2):  # a second call on the cached workspace, the previous argmax as argmax_prev
         fused = dg.dg_sampler_step_eb(logits, cfg.C, eps=40.0, theta=6.0, argmax_prev=prev, inv_tau=inv_tau, seed=7,
                                       step=5 + rep)
         torch.cuda.synchronize()
